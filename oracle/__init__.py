@@ -1,0 +1,192 @@
+"""CPU oracle of the NVFP4 quantized linear layer (binding to fh_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline / reference legs may import this package.  It shares
+no code with the CUDA library and imports nothing from it.
+
+Every function states the definition it computes; fh_oracle.c carries the
+citations (FastH3 thread digest, farwalk.ai, tweets 5/8 and 6/8; FastH3 Trim,
+comfyui-wiki news, "What the ComfyUI repack contains").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "fh_oracle.c")
+_LIB = os.path.join(_HERE, "libfh_oracle.so")
+
+#: Largest magnitude of the scaled format: 6 (E2M1) * 448 (E4M3).
+FORMAT_MAX = 2688.0
+
+
+def build(force: bool = False) -> str:
+    """Compile fh_oracle.c with gcc (plain -O2, OpenMP, no FMA contraction)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+               "-shared", "-fPIC", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        c = ctypes
+        L.oracle_bf16_value.restype = c.c_double
+        L.oracle_bf16_value.argtypes = [c.c_uint16]
+        L.oracle_e2m1_value.restype = c.c_double
+        L.oracle_e2m1_value.argtypes = [c.c_int]
+        L.oracle_e4m3_value.restype = c.c_double
+        L.oracle_e4m3_value.argtypes = [c.c_int]
+        L.oracle_e4m3_rne_sat.restype = c.c_int
+        L.oracle_e4m3_rne_sat.argtypes = [c.c_double]
+        L.oracle_e2m1_rne_sat.restype = c.c_int
+        L.oracle_e2m1_rne_sat.argtypes = [c.c_double]
+        L.oracle_scale_from_amax.restype = c.c_float
+        L.oracle_scale_from_amax.argtypes = [c.c_float]
+        L.oracle_amax.restype = c.c_float
+        L.oracle_amax.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_int64]
+        L.oracle_quantize.restype = None
+        L.oracle_quantize.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_int64, c.c_float,
+                                      c.c_void_p, c.c_void_p, c.c_void_p]
+        L.oracle_linear.restype = None
+        L.oracle_linear.argtypes = [c.c_void_p, c.c_void_p, c.c_float, c.c_void_p, c.c_void_p, c.c_float,
+                                    c.c_void_p, c.c_int64, c.c_int64, c.c_void_p, c.c_int64,
+                                    c.c_void_p, c.c_void_p, c.c_void_p, c.c_void_p]
+        L.oracle_gelu.restype = None
+        L.oracle_gelu.argtypes = [c.c_void_p, c.c_int64, c.c_void_p]
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+# --- element formats --------------------------------------------------------
+
+def bf16_value(bits: int) -> float:
+    return lib().oracle_bf16_value(bits)
+
+
+def e2m1_value(code: int) -> float:
+    """Value of a 4-bit E2M1 code (bit 3 sign; magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6)."""
+    return lib().oracle_e2m1_value(code)
+
+
+def e4m3_value(byte: int) -> float:
+    """Value of an E4M3 (FN) byte; NaN for 0x7F / 0xFF."""
+    return lib().oracle_e4m3_value(byte)
+
+
+def e4m3_rne_sat(q: float) -> int:
+    """E4M3 code of q >= 0: nearest, ties to even, q >= 448 gives 448."""
+    return lib().oracle_e4m3_rne_sat(q)
+
+
+def e2m1_rne_sat(r: float) -> int:
+    """E2M1 magnitude code of r >= 0: nearest, ties to even, saturating at 6."""
+    return lib().oracle_e2m1_rne_sat(r)
+
+
+# --- calibration -------------------------------------------------------------
+
+def scale_from_amax(amax: float) -> float:
+    """Smallest FP32 s_g with 2688 * s_g >= amax (1.0 for amax == 0)."""
+    return lib().oracle_scale_from_amax(float(amax))
+
+
+def amax(x_bits: np.ndarray) -> float:
+    """max |x| over a BF16 matrix given as uint16 bits [rows, cols]."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    return lib().oracle_amax(_ptr(x), x.shape[0], x.shape[1], x.shape[1])
+
+
+# --- quantization ----------------------------------------------------------
+
+def quantize(x_bits: np.ndarray, sg: float):
+    """Quantize BF16 x [M, K] (K % 16 == 0) with global scale sg.
+
+    Returns (codes [M, K/2] uint8 with element 2j in the low nibble,
+             scales [M, K/16] uint8 E4M3, row-major,
+             clip count: elements with |x| > 2688 * sg)."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    M, K = x.shape
+    assert K % 16 == 0
+    codes = np.empty((M, K // 2), dtype=np.uint8)
+    scales = np.empty((M, K // 16), dtype=np.uint8)
+    clip = np.zeros(1, dtype=np.uint64)
+    lib().oracle_quantize(_ptr(x), M, K, K, float(sg), _ptr(codes), _ptr(scales), _ptr(clip))
+    return codes, scales, int(clip[0])
+
+
+def tiled_scale_offsets(rows: int, K: int) -> np.ndarray:
+    """Byte offset, in the tensor-core (MMA-tiled) scale layout, of scale (r, s)
+    for r < rows, s < K/16.
+
+    The layout is the one the block-scaled tensor-core MMA reads: rows are
+    padded to a multiple of 128 and scale columns to a multiple of 4; the
+    matrix is cut into atoms of 128 rows x 4 scales (512 bytes), atoms ordered
+    with the K-atom index fastest; inside an atom, row r = r0 + 32 r1
+    (r0 < 32, r1 < 4) and scale column s = 4 k1 + k0 sit at byte
+    r0 * 16 + r1 * 4 + k0."""
+    ns = K // 16
+    ka = -(-ns // 4)
+    r = np.arange(rows)[:, None]
+    s = np.arange(ns)[None, :]
+    atom = (r // 128) * ka + s // 4
+    rr = r % 128
+    return atom * 512 + (rr % 32) * 16 + (rr // 32) * 4 + s % 4
+
+
+def tiled_scales_bytes(rows: int, K: int) -> int:
+    return (-(-rows // 128)) * 128 * (-(-(K // 16) // 4)) * 4
+
+
+# --- linear layer ------------------------------------------------------------
+
+def linear(a_codes, a_scales, a_g, w_codes, w_scales, w_g, bias_bits, rows=None):
+    """y = a_g * w_g * (A_deq . W_deq^T) + bias in binary64, on the requested rows.
+
+    Returns (y [len(rows), N], mag [len(rows), N]) where mag is
+    |a_g * w_g| * sum_k |A_deq[m,k] * W_deq[n,k]| (the error-bound magnitude)."""
+    a_codes = np.ascontiguousarray(a_codes, dtype=np.uint8)
+    a_scales = np.ascontiguousarray(a_scales, dtype=np.uint8)
+    w_codes = np.ascontiguousarray(w_codes, dtype=np.uint8)
+    w_scales = np.ascontiguousarray(w_scales, dtype=np.uint8)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    rows = np.arange(M, dtype=np.int64) if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits, dtype=np.uint16)
+    y = np.empty((rows.size, N), dtype=np.float64)
+    mag = np.empty((rows.size, N), dtype=np.float64)
+    w_deq = np.empty((N, K), dtype=np.float64)
+    a_deq = np.empty((rows.size, K), dtype=np.float64)
+    lib().oracle_linear(_ptr(a_codes), _ptr(a_scales), float(a_g), _ptr(w_codes), _ptr(w_scales), float(w_g),
+                        None if b is None else _ptr(b), N, K, _ptr(rows), rows.size,
+                        _ptr(w_deq), _ptr(a_deq), _ptr(y), _ptr(mag))
+    return y, mag
+
+
+def linear_tolerance(y_ref: np.ndarray, mag: np.ndarray) -> np.ndarray:
+    """Allowed |y - y_ref| of a BF16 output: 2^-8 |y_ref| + 1e-5 * mag."""
+    return np.abs(y_ref) * 2.0 ** -8 + 1e-5 * mag
+
+
+def gelu(x_bits: np.ndarray) -> np.ndarray:
+    """Exact-erf GELU of BF16 inputs, in binary64."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16).reshape(-1)
+    y = np.empty(x.size, dtype=np.float64)
+    lib().oracle_gelu(_ptr(x), x.size, _ptr(y))
+    return y.reshape(np.shape(x_bits))
