@@ -1,0 +1,330 @@
+"""Benchmark of the NVFP4 quantized linear layer on B200.
+
+One step = one pass of the whole hot path over one batch: NVFP4 quantization
+of the BF16 activations with the layer's calibrated scale (fh_quantize_act)
+followed by the block-scaled tensor-core GEMM with its fused epilogue
+(fh_nvfp4_linear), on the fused-QKV workload of the transformer (FastH3 Trim,
+comfyui-wiki news: hidden width 2688): M = 32768 tokens, K = 2688, N = 8064.
+The calibration, the weight quantization and the input generation happen
+before the timed region.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fh|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs the same
+per-GPU workload on its own GPU (rows of the token batch are independent:
+weak scaling, no data-path collective); the time is the max over ranks.
+--impl reference times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 linear TFLOPS (M×2688→N) and % of B200 FP4 peak; quantizer GB/s"
+WORKLOAD = {"name": "qkv", "M": 32768, "K": 2688, "N": 8064}
+FP4_OVER_BF16 = 4.0        # nominal dense ratio 9 / 2.25 PFLOP/s
+QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16.0
+CPU_SAMPLE_ROWS = 64
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def make_inputs(rank: int):
+    """Seeded synthetic fused-QKV layer (channel std log-normal, calibration over
+    1000 batches of 64 tokens whose first 512 form the input)."""
+    import synthetic as S
+    layer = S.workloads()["qkv"][0]
+    if rank:
+        layer = S.Layer(layer.name, layer.M, layer.K, layer.N, layer.batch, layer.n_calib,
+                        channel_lognormal=True, key=("qkv", rank))
+    return S, layer
+
+
+def bench_fh(args, rank, world, local_rank):
+    import torch
+    import nvfp4_quantized_linear_fh_b200 as fh
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    S, layer = make_inputs(rank)
+    M, K, N = layer.M, layer.K, layer.N
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    # --- offline: calibration, weight quantization (not timed) ---
+    x_bits = S.activations(layer)
+    x = to_dev(x_bits)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    fh.fh_amax(x, amax)
+    chunk = 64
+    for b0 in range(layer.n_eval_batches, layer.n_calib, chunk):
+        nb = min(chunk, layer.n_calib - b0)
+        fh.fh_amax(to_dev(S.activation_batches(layer, b0, nb)), amax)
+    sg_a = fh.fh_scale_from_amax(amax.item())
+    w = to_dev(S.weights(layer))
+    wamax = torch.zeros(1, dtype=torch.float32, device=dev)
+    fh.fh_amax(w, wamax)
+    sg_w = fh.fh_scale_from_amax(wamax.item())
+    wc, wsc = fh.empty_quantized(N, K, device=dev)
+    fh.fh_quantize_act(w, sg_w, wc, wsc, None)
+    bias = to_dev(S.bias(layer))
+    del w
+
+    ac, asc = fh.empty_quantized(M, K, device=dev)
+    clip = torch.zeros(1, dtype=torch.int64, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)  # > L2 (126 MB)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fh.fh_quantize_act(x, sg_a, ac, asc, clip)
+        fh.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, bias, y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clip.zero_()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else local_rank)
+    with sampler:
+        for i in range(args.steps):
+            flush.fill_(i)                      # evict the previous step's data from L2
+            ev[i][0].record(stream)
+            fh.fh_quantize_act(x, sg_a, ac, asc, clip)
+            ev[i][1].record(stream)
+            fh.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, bias, y)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t_quant = [ev[i][0].elapsed_time(ev[i][1]) * 1e-3 for i in range(args.steps)]
+    t_gemm = [ev[i][1].elapsed_time(ev[i][2]) * 1e-3 for i in range(args.steps)]
+    t_step = sum(t_quant) + sum(t_gemm)
+    fh.fh_device_status()
+    clips = int(clip.item())
+
+    # --- end to end through the public API with host buffers ---
+    x_host = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(x.cpu())
+    y_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    x_stage = torch.empty_like(x)
+    e_steps = max(2, min(args.steps, 5))
+    for _ in range(2):
+        x_stage.copy_(x_host, non_blocking=True)
+        fh.fh_quantize_act(x_stage, sg_a, ac, asc, None)
+        fh.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, bias, y)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    e0.record(stream)
+    for _ in range(e_steps):
+        x_stage.copy_(x_host, non_blocking=True)
+        fh.fh_quantize_act(x_stage, sg_a, ac, asc, None)
+        fh.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, bias, y)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t_e2e = e0.elapsed_time(e1) * 1e-3
+
+    if world > 1:
+        t = torch.tensor([t_step, t_e2e, max(t_gemm), max(t_quant)], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_step, t_e2e = float(t[0]), float(t[1])
+    flops = 2.0 * M * N * K
+    return dict(t_step=t_step, t_quant=t_quant, t_gemm=t_gemm, t_e2e=t_e2e, e_steps=e_steps, flops=flops,
+                clips=clips, sampler=sampler.summary(), M=M, N=N, K=K,
+                h2d=M * K * 2, d2h=M * N * 2, x_bits=x_bits, w_bits=S.weights(layer), b_bits=S.bias(layer),
+                sg_a=sg_a, sg_w=sg_w)
+
+
+def cpu_baseline(x_bits, w_bits, b_bits, sg_a, sg_w, rows):
+    """The oracle, as it stands, on the first `rows` rows: quantize them, quantize
+    the weights, binary64 dequantized product.  Returns (TFLOPS, seconds, cores)."""
+    import oracle
+    oracle.build()
+    K, N = x_bits.shape[1], w_bits.shape[0]
+    t0 = time.perf_counter()
+    ac, asc, _ = oracle.quantize(x_bits[:rows], sg_a)
+    wc, wsc, _ = oracle.quantize(w_bits, sg_w)
+    oracle.linear(ac, asc, sg_a, wc, wsc, sg_w, b_bits)
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return 2.0 * rows * N * K / dt / 1e12, dt, cores
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="fh", choices=["fh", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    pk = peaks()
+    cfg = {"workload": f"fused QKV linear {WORKLOAD['M']}x{WORKLOAD['K']}->{WORKLOAD['N']} (M x K -> N) per GPU",
+           "M": WORKLOAD["M"], "K": WORKLOAD["K"], "N": WORKLOAD["N"], "tokens_per_gpu": WORKLOAD["M"],
+           "parallelism": f"dp{world} (token rows per GPU, replicas)", "l2": "flushed between steps (256 MB write)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import synthetic as S
+        layer = S.workloads()["qkv"][0]
+        x_bits = S.activation_batches(layer, 0, 1)
+        w_bits, b_bits = S.weights(layer), S.bias(layer)
+        import oracle
+        sg_a = oracle.scale_from_amax(oracle.amax(x_bits))
+        sg_w = oracle.scale_from_amax(oracle.amax(w_bits))
+        vals, secs = [], []
+        for i in range(args.warmup + args.steps):
+            v, dt, cores = cpu_baseline(x_bits, w_bits, b_bits, sg_a, sg_w, 8)
+            if i >= args.warmup:
+                vals.append(v)
+                secs.append(dt)
+        value = statistics.median(vals)
+        sample = "8 token rows of the fused-QKV layer per step (quantize rows + weights, binary64 GEMM)"
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+                          "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": statistics.median(secs) * 1e3, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": cfg,
+                          "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                                           "sample": sample},
+                          "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}))
+        return
+
+    import torch
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    r = bench_fh(args, rank, world, local_rank)
+    K_steps = args.steps
+    value = r["flops"] * K_steps * world / r["t_step"] / 1e12
+    gemm_mean = statistics.mean(r["t_gemm"])
+    quant_mean = statistics.mean(r["t_quant"])
+    achieved = r["flops"] / gemm_mean / 1e12
+    fp4_sust = pk["bf16_sustained"] * FP4_OVER_BF16
+    fp4_burst = pk["bf16"] * FP4_OVER_BF16
+    quant_gbs = QUANT_BYTES_PER_ELEM * r["M"] * r["K"] / quant_mean / 1e9
+    e2e_value = r["flops"] * r["e_steps"] * world / r["t_e2e"] / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K_steps,
+        "warmup": args.warmup, "ms_per_step": r["t_step"] / K_steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e4m3, fp32 accumulate, bf16 out)",
+        "data": "synthetic (seeded; calibrated per-layer scale; random-init weights)", "config": cfg,
+        "gpu_launches": 2 * K_steps,
+        "roofline": {"kernel": "nvfp4_linear_kernel", "bound": "tensor", "achieved": achieved,
+                     "peak": fp4_sust, "unit": "TFLOP/s", "frac": achieved / fp4_sust,
+                     "peak_note": f"{pk['source']} bf16 sustained {pk['bf16_sustained']} x 4 (nominal FP4/BF16)",
+                     "frac_of_burst_peak": achieved / fp4_burst, "traffic": None},
+        "quantizer": {"kernel": "quantize_kernel", "bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"],
+                      "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"], "us": quant_mean * 1e6},
+        "gemm_us": gemm_mean * 1e6, "clip_count": r["clips"],
+        "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "steps": r["e_steps"]},
+        "clocks": r["sampler"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, cores = cpu_baseline(r["x_bits"], r["w_bits"], r["b_bits"], r["sg_a"], r["sg_w"], CPU_SAMPLE_ROWS)
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                                "sample": f"first {CPU_SAMPLE_ROWS} token rows of the same layer "
+                                          f"(quantize rows + weights, binary64 GEMM), {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,156 @@
+/*
+ * fh.h -- C ABI of the NVFP4 quantized linear layer for B200 (sm_100a).
+ *
+ * The layer is the FP4 linear layer that FastH3 runs inside every block of its
+ * diffusion transformer:
+ *   - FastH3 thread digest (farwalk.ai), tweet 5/8: on Blackwell the
+ *     transformer runs in NVFP4;
+ *   - FastH3 thread digest (farwalk.ai), tweet 6/8: every FP4 layer is
+ *     calibrated on 1,000 prompts so that large activations are not clipped,
+ *     where uncalibrated FP4 scales clip in 40 of 42 blocks (worst 137x);
+ *   - FastH3 Trim (comfyui-wiki news), "What the ComfyUI repack contains":
+ *     each NVFP4 layer carries an activation scale calibrated on 1,000
+ *     prompts, 294 calibrated layers in all;
+ *   - FastH3 Trim (comfyui-wiki news), "Trim changes": the transformer's
+ *     hidden width is 2,688.
+ *
+ * NVFP4 (the pages name it without defining it; this is the public format):
+ * a tensor x is stored as 4-bit E2M1 codes (magnitudes 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6; bit 3 the sign), one unsigned E4M3 block scale S_b per 16 consecutive
+ * elements along K, and one FP32 global scale s_g, with x ~ code * S_b * s_g.
+ * Rounding is to nearest, ties to the even code, on the exact quotients
+ * (S_b = E4M3(amax_b / (6 s_g)), saturating at 448; code = E2M1(x / (S_b s_g)),
+ * saturating at 6; the code's sign bit is always the sign bit of x).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_dev or documented as device pointers are device memory
+ *     owned by the caller; the library allocates nothing and keeps no state
+ *     between calls except a per-device property cache and one device error
+ *     word.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream) and the call returns without synchronizing, except where stated.
+ *   - The return value is an fh_status.  On failure nothing was enqueued and
+ *     fh_last_error() (per host thread) describes the cause.
+ *   - Matrices are row-major.  BF16 values are passed as their uint16 bits.
+ *   - Inputs must be finite; results for NaN or Inf inputs are unspecified.
+ */
+#ifndef FH_H_
+#define FH_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fh_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  FH_OK = 0,
+  FH_ERR_INVALID_ARG = 1,       /* null pointer, bad enum, non-finite or <= 0 scale */
+  FH_ERR_UNSUPPORTED_SHAPE = 2, /* a size or alignment rule below is violated */
+  FH_ERR_CUDA = 3,              /* a CUDA call failed; fh_last_error() has its text */
+  FH_ERR_TIMEOUT = 4,           /* a bounded on-chip wait expired (see fh_device_status) */
+  FH_ERR_NO_DEVICE = 5          /* the current device is not an sm_100 GPU */
+} fh_status;
+
+/* Scale layouts accepted by fh_quantize_act. */
+enum {
+  /* scales[r * (K/16) + s]: plain row-major [rows, K/16]. */
+  FH_SCALES_ROWMAJOR = 0,
+  /* The layout the block-scaled tensor-core MMA reads (fh_nvfp4_linear's
+   * operand layout).  Rows are padded to a multiple of 128 and K/16 to a
+   * multiple of 4.  The matrix is cut into 512-byte atoms of 128 rows x 4
+   * scales; atom (r/128, s/4) sits at ((r/128) * ceil(K/64) + s/4) * 512;
+   * inside it, row r%128 = r0 + 32*r1 and scale s%4 = k0 sit at byte
+   * r0*16 + r1*4 + k0.  Padding rows hold zero scales. */
+  FH_SCALES_MMA_TILED = 1
+};
+
+/* Library version, as major*10000 + minor*100 + patch. */
+int fh_version(void);
+
+/* Text of the last failure on this host thread ("" if none). */
+const char* fh_last_error(void);
+
+/* Global scale from a calibrated amax (host only, no GPU needed).
+ * Calibration maps the amax seen over the calibration set onto the largest
+ * magnitude of the scaled format, 6 * 448 = 2688, so that no calibrated
+ * activation clips (FastH3 thread digest, tweet 6/8).  Returns the SMALLEST
+ * FP32 s_g with 2688 * s_g >= amax; amax == 0 gives 1.0; a negative or
+ * non-finite amax gives NaN. */
+float fh_scale_from_amax(float amax);
+
+/* Bytes of the scale array of a quantized [rows, K] matrix in `layout`
+ * (0 for an invalid layout or size). */
+size_t fh_scales_bytes(int64_t rows, int64_t K, int layout);
+
+/* Running max |x| over a BF16 matrix x [rows, cols] (leading dimension ldx >=
+ * cols, in elements), merged into *amax_dev (device float, caller initialises
+ * it, e.g. to 0): *amax_dev = max(*amax_dev, max |x|).  Calling it once per
+ * calibration batch gives the calibrated amax (FastH3 thread digest, tweet
+ * 6/8).  Exact (a max), deterministic.  rows == 0 or cols == 0 enqueues
+ * nothing.  Requires 0 <= rows, cols and ldx >= cols. */
+int fh_amax(const uint16_t* x_dev, int64_t rows, int64_t cols, int64_t ldx,
+            float* amax_dev, fh_stream_t stream);
+
+/* NVFP4 quantization of BF16 activations (or weights) x [M, K] (leading
+ * dimension ldx >= K, elements) with the calibrated global scale s_g
+ * (FastH3 Trim, "What the ComfyUI repack contains": per-layer calibrated
+ * activation scale).
+ * Outputs (device memory, caller-allocated):
+ *   codes       [M, K/2] bytes; element 2j of a row in the low nibble of byte j.
+ *   scales      E4M3 block scales in `scale_layout`
+ *               (fh_scales_bytes(M, K, scale_layout) bytes).
+ *   clip_count  device counter, INCREMENTED by the number of elements with
+ *               |x| > 2688 * s_g (beyond the largest magnitude the scaled
+ *               format holds; FastH3 thread digest, tweet 6/8); may be NULL.
+ * Requires: M >= 0, K > 0, K % 16 == 0 (K % 64 == 0 for FH_SCALES_MMA_TILED),
+ * ldx >= K and ldx % 8 == 0, x_dev and codes_dev 16-byte aligned, s_g finite
+ * and > 0.  Results are bit-exact with the rounding rules in the header
+ * comment.  M == 0 only pads nothing and enqueues nothing. */
+int fh_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx,
+                    float global_scale, uint8_t* codes_dev, uint8_t* scales_dev,
+                    unsigned long long* clip_count_dev, int scale_layout,
+                    fh_stream_t stream);
+
+/* NVFP4 linear layer on the tcgen05 tensor cores (FastH3 thread digest, tweet
+ * 5/8: the transformer's linear layers in NVFP4 on Blackwell):
+ *   y[m, n] = bf16( a_gscale * w_gscale * sum_k A[m,k] * W[n,k] + bias[n] )
+ * where A[m,k] = E2M1(a_codes) * E4M3(a_scales) and W likewise, both K-major
+ * (W is [N, K], the usual nn.Linear weight), the block products are summed in
+ * FP32 on the tensor cores, and the epilogue is one FP32 fma then a
+ * round-to-nearest-even BF16 store.
+ *   a_codes  [M, K/2], a_scales FH_SCALES_MMA_TILED of [M, K]
+ *   w_codes  [N, K/2], w_scales FH_SCALES_MMA_TILED of [N, K]
+ *   bias     [N] BF16 or NULL; y [M, N] BF16 (row stride N).
+ * Requires: M, N >= 0, K > 0, K % 64 == 0, N % 8 == 0, all pointers 16-byte
+ * aligned, scales finite and > 0.  M == 0 or N == 0 enqueues nothing.
+ * A bounded wait that expires inside the kernel sets the device error word
+ * (see fh_device_status) instead of hanging. */
+int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, float a_gscale,
+                    const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                    const uint16_t* bias_dev, uint16_t* y_dev, int64_t M, int64_t N,
+                    int64_t K, fh_stream_t stream);
+
+/* Permute FH_SCALES_MMA_TILED scales of a [rows, K] matrix into row-major
+ * [rows, K/16] (drops the padding).  Requires K % 64 == 0. */
+int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows,
+                          int64_t K, fh_stream_t stream);
+
+/* Exact-erf GELU on BF16, y = bf16(x/2 * (1 + erf(x/sqrt 2))) computed in
+ * FP32; the activation between the two linear layers of the FFN.  n >= 0;
+ * x_dev and y_dev 16-byte aligned; in-place (x_dev == y_dev) is allowed. */
+int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t stream);
+
+/* Synchronizes `stream`, then reads and clears the device error word of the
+ * current device.  Returns FH_OK, FH_ERR_TIMEOUT if a kernel gave up on a
+ * bounded wait since the last call, or FH_ERR_CUDA. */
+int fh_device_status(fh_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FH_H_ */

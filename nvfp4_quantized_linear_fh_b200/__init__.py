@@ -1,0 +1,203 @@
+"""Python binding of libfh, the NVFP4 quantized linear layer for B200 (sm_100a).
+
+Argument marshalling only: every function below has the name of the C entry
+point it calls (include/fh.h), checks that the torch tensors it is given have
+the dtype, device and contiguity the C ABI expects, passes their device
+pointers and the current CUDA stream, and raises FHError on a non-zero status.
+All arithmetic runs in the CUDA kernels of libfh.so.  There is no fallback:
+importing this package fails if libfh.so has not been built
+(``python nvfp4_quantized_linear_fh_b200/build.py``).
+
+The layer is the NVFP4 linear layer of FastH3's diffusion transformer (FastH3
+thread digest, farwalk.ai, tweets 5/8 and 6/8; FastH3 Trim, comfyui-wiki news,
+"What the ComfyUI repack contains").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfh.so")
+
+FH_OK = 0
+FH_ERR_INVALID_ARG = 1
+FH_ERR_UNSUPPORTED_SHAPE = 2
+FH_ERR_CUDA = 3
+FH_ERR_TIMEOUT = 4
+FH_ERR_NO_DEVICE = 5
+
+FH_SCALES_ROWMAJOR = 0
+FH_SCALES_MMA_TILED = 1
+
+
+class FHError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"libfh status {status}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python nvfp4_quantized_linear_fh_b200/build.py` "
+                      "(the NVFP4 layer has no CPU fallback)")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_c = ctypes
+_P = _c.c_void_p
+_I64 = _c.c_int64
+_SIG = {
+    "fh_version": (_c.c_int, []),
+    "fh_last_error": (_c.c_char_p, []),
+    "fh_scale_from_amax": (_c.c_float, [_c.c_float]),
+    "fh_scales_bytes": (_c.c_size_t, [_I64, _I64, _c.c_int]),
+    "fh_amax": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P]),
+    "fh_quantize_act": (_c.c_int, [_P, _I64, _I64, _I64, _c.c_float, _P, _P, _P, _c.c_int, _P]),
+    "fh_nvfp4_linear": (_c.c_int, [_P, _P, _c.c_float, _P, _P, _c.c_float, _P, _P, _I64, _I64, _I64, _P]),
+    "fh_scales_to_rowmajor": (_c.c_int, [_P, _P, _I64, _I64, _P]),
+    "fh_gelu_bf16": (_c.c_int, [_P, _P, _I64, _P]),
+    "fh_device_status": (_c.c_int, [_P]),
+}
+for _name, (_res, _args) in _SIG.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def lib():
+    """The loaded ctypes library (for tests that call the C ABI directly)."""
+    return _lib
+
+
+def _check(status: int):
+    if status != FH_OK:
+        raise FHError(status, _lib.fh_last_error().decode())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return _P(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else _P(t.data_ptr())
+
+
+def _need(t, dtypes, what, ndim=None):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cuda":
+        raise TypeError(f"{what} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{what} must have dtype in {dtypes}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{what} must have {ndim} dimensions")
+
+
+_BF16 = (torch.bfloat16, torch.int16, torch.uint16)
+_U8 = (torch.uint8,)
+
+
+# --- host entry points --------------------------------------------------------
+
+def fh_version() -> int:
+    return _lib.fh_version()
+
+
+def fh_last_error() -> str:
+    return _lib.fh_last_error().decode()
+
+
+def fh_scale_from_amax(amax: float) -> float:
+    return _lib.fh_scale_from_amax(float(amax))
+
+
+def fh_scales_bytes(rows: int, K: int, layout: int = FH_SCALES_MMA_TILED) -> int:
+    return _lib.fh_scales_bytes(rows, K, layout)
+
+
+# --- device entry points ------------------------------------------------------
+
+def fh_amax(x: torch.Tensor, amax: torch.Tensor, stream=None) -> None:
+    """amax[0] = max(amax[0], max |x|) for BF16 x [rows, cols] (row stride x.stride(0))."""
+    _need(x, _BF16, "x", 2)
+    _need(amax, (torch.float32,), "amax")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit column stride")
+    _check(_lib.fh_amax(_ptr(x), x.shape[0], x.shape[1], x.stride(0), _ptr(amax), _stream(stream)))
+
+
+def fh_quantize_act(x: torch.Tensor, global_scale: float, codes: torch.Tensor, scales: torch.Tensor,
+                    clip_count: torch.Tensor | None = None, scale_layout: int = FH_SCALES_MMA_TILED,
+                    stream=None) -> None:
+    """NVFP4-quantize BF16 x [M, K] into codes [M, K/2] and scales (see include/fh.h)."""
+    _need(x, _BF16, "x", 2)
+    _need(codes, _U8, "codes")
+    _need(scales, _U8, "scales")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit column stride")
+    M, K = x.shape
+    if codes.numel() < M * (K // 2) or not codes.is_contiguous():
+        raise ValueError("codes must be contiguous with M*K/2 bytes")
+    need = fh_scales_bytes(M, K, scale_layout)
+    if scales.numel() < need or not scales.is_contiguous():
+        raise ValueError(f"scales must be contiguous with {need} bytes")
+    if clip_count is not None:
+        _need(clip_count, (torch.int64, torch.uint64), "clip_count")
+    _check(_lib.fh_quantize_act(_ptr(x), M, K, x.stride(0), float(global_scale), _ptr(codes), _ptr(scales),
+                                _ptr(clip_count), scale_layout, _stream(stream)))
+
+
+def fh_nvfp4_linear(a_codes: torch.Tensor, a_scales: torch.Tensor, a_gscale: float,
+                    w_codes: torch.Tensor, w_scales: torch.Tensor, w_gscale: float,
+                    bias: torch.Tensor | None, y: torch.Tensor, stream=None) -> None:
+    """y[M, N] = bf16(a_g * w_g * A . W^T + bias) on the tcgen05 tensor cores."""
+    for t, n in ((a_codes, "a_codes"), (w_codes, "w_codes")):
+        _need(t, _U8, n, 2)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_scales, _U8, "a_scales")
+    _need(w_scales, _U8, "w_scales")
+    _need(y, _BF16, "y", 2)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K or tuple(y.shape) != (M, N) or not y.is_contiguous():
+        raise ValueError("shape mismatch: a_codes [M, K/2], w_codes [N, K/2], y [M, N] contiguous")
+    if a_scales.numel() < fh_scales_bytes(M, K) or w_scales.numel() < fh_scales_bytes(N, K):
+        raise ValueError("scale arrays too small for the tensor-core scale layout")
+    if bias is not None:
+        _need(bias, _BF16, "bias")
+        if bias.numel() != N or not bias.is_contiguous():
+            raise ValueError("bias must be contiguous with N elements")
+    _check(_lib.fh_nvfp4_linear(_ptr(a_codes), _ptr(a_scales), float(a_gscale), _ptr(w_codes), _ptr(w_scales),
+                                float(w_gscale), _ptr(bias), _ptr(y), M, N, K, _stream(stream)))
+
+
+def fh_scales_to_rowmajor(tiled: torch.Tensor, rowmajor: torch.Tensor, rows: int, K: int, stream=None) -> None:
+    _need(tiled, _U8, "tiled")
+    _need(rowmajor, _U8, "rowmajor")
+    if rowmajor.numel() < rows * (K // 16) or tiled.numel() < fh_scales_bytes(rows, K):
+        raise ValueError("buffer too small")
+    _check(_lib.fh_scales_to_rowmajor(_ptr(tiled), _ptr(rowmajor), rows, K, _stream(stream)))
+
+
+def fh_gelu_bf16(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    _need(x, _BF16, "x")
+    _need(y, _BF16, "y")
+    if x.numel() != y.numel() or not x.is_contiguous() or not y.is_contiguous():
+        raise ValueError("x and y must be contiguous with the same number of elements")
+    _check(_lib.fh_gelu_bf16(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+
+
+def fh_device_status(stream=None) -> None:
+    """Synchronize and raise FHError(FH_ERR_TIMEOUT) if a kernel gave up on a bounded wait."""
+    _check(_lib.fh_device_status(_stream(stream)))
+
+
+# --- allocation helpers (marshalling only) ----------------------------------------
+
+def empty_quantized(rows: int, K: int, device="cuda", layout: int = FH_SCALES_MMA_TILED):
+    """Uninitialised (codes [rows, K/2], scales) buffers for fh_quantize_act."""
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty(max(fh_scales_bytes(rows, K, layout), 1), dtype=torch.uint8, device=device)
+    return codes, scales

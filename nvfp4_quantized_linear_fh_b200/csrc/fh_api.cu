@@ -1,0 +1,194 @@
+// fh_api.cu -- the extern "C" entry points declared in include/fh.h: argument
+// validation, error reporting and dispatch to the kernels.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "fh_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, const char* detail = nullptr) {
+  snprintf(g_last_error, sizeof g_last_error, fmt, detail ? detail : "");
+  return status;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof g_last_error, "%s: %s", where, cudaGetErrorString(e));
+  return FH_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device checks shared by every entry point: a current device of compute
+// capability 10.0 (B200 class).  Cached per device.
+int check_device() {
+  static int checked_dev = -1;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev == checked_dev) return FH_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0)
+    return fail(FH_ERR_NO_DEVICE, "current device is not an sm_100 GPU%s");
+  checked_dev = dev;
+  return FH_OK;
+}
+
+}  // namespace
+
+namespace fh {
+
+int sm_count() {
+  static int dev_cached = -1, count = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != dev_cached) {
+    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+    dev_cached = dev;
+  }
+  return count > 0 ? count : 1;
+}
+
+}  // namespace fh
+
+extern "C" {
+
+int fh_version(void) { return 10000; }
+
+const char* fh_last_error(void) { return g_last_error; }
+
+float fh_scale_from_amax(float amax) {
+  if (!(amax >= 0.0f) || isinf(amax)) return NAN;
+  if (amax == 0.0f) return 1.0f;
+  const double target = (double)amax;
+  // Start from the nearest FP32 to amax / 2688, then move to the smallest FP32
+  // whose product with 2688 (exact in FP64) still covers amax.
+  float s = (float)(target / 2688.0);
+  while ((double)s * 2688.0 < target) s = nextafterf(s, INFINITY);
+  for (;;) {
+    const float below = nextafterf(s, 0.0f);
+    if (below <= 0.0f || (double)below * 2688.0 < target) break;
+    s = below;
+  }
+  return s;
+}
+
+size_t fh_scales_bytes(int64_t rows, int64_t K, int layout) {
+  if (rows < 0 || K <= 0 || K % 16 != 0) return 0;
+  if (layout == FH_SCALES_ROWMAJOR) return (size_t)rows * (size_t)(K / 16);
+  if (layout == FH_SCALES_MMA_TILED) {
+    if (K % 64 != 0) return 0;
+    return (size_t)((rows + 127) / 128) * 128 * (size_t)(K / 16);
+  }
+  return 0;
+}
+
+int fh_amax(const uint16_t* x_dev, int64_t rows, int64_t cols, int64_t ldx, float* amax_dev,
+            fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (rows < 0 || cols < 0 || ldx < cols)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_amax: need rows, cols >= 0 and ldx >= cols%s");
+  if (amax_dev == nullptr || (x_dev == nullptr && rows * cols > 0))
+    return fail(FH_ERR_INVALID_ARG, "fh_amax: null pointer%s");
+  if (rows == 0 || cols == 0) return FH_OK;
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_amax(x_dev, rows, cols, ldx, amax_dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_amax launch");
+}
+
+int fh_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx, float global_scale,
+                    uint8_t* codes_dev, uint8_t* scales_dev, unsigned long long* clip_count_dev,
+                    int scale_layout, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (scale_layout != FH_SCALES_ROWMAJOR && scale_layout != FH_SCALES_MMA_TILED)
+    return fail(FH_ERR_INVALID_ARG, "fh_quantize_act: unknown scale layout%s");
+  if (!(global_scale > 0.0f) || isinf(global_scale))
+    return fail(FH_ERR_INVALID_ARG, "fh_quantize_act: global scale must be finite and > 0%s");
+  if (M < 0 || K <= 0 || K % 16 != 0 || ldx < K || ldx % 8 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_quantize_act: need M >= 0, K > 0, K %% 16 == 0, ldx >= K, ldx %% 8 == 0%s");
+  if (scale_layout == FH_SCALES_MMA_TILED && K % 64 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_quantize_act: the tensor-core scale layout needs K %% 64 == 0%s");
+  if (M == 0) return FH_OK;
+  if (x_dev == nullptr || codes_dev == nullptr || scales_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_quantize_act: null pointer%s");
+  if (!aligned16(x_dev) || !aligned16(codes_dev) || !aligned16(scales_dev))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_quantize_act: x, codes and scales must be 16-byte aligned%s");
+  if (M * (K / 16) > ((int64_t)1 << 40))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_quantize_act: tensor too large%s");
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_quantize(x_dev, M, K, ldx, global_scale, codes_dev, scales_dev, clip_count_dev,
+                                      scale_layout, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_quantize_act launch");
+}
+
+int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, float a_gscale,
+                    const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                    const uint16_t* bias_dev, uint16_t* y_dev, int64_t M, int64_t N, int64_t K,
+                    fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!(a_gscale > 0.0f) || isinf(a_gscale) || !(w_gscale > 0.0f) || isinf(w_gscale))
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear: global scales must be finite and > 0%s");
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || N % 8 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear: need M, N >= 0, K > 0, K %% 64 == 0, N %% 8 == 0%s");
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear: each dimension must fit in 31 bits%s");
+  if (M == 0 || N == 0) return FH_OK;
+  if (a_codes_dev == nullptr || a_scales_dev == nullptr || w_codes_dev == nullptr || w_scales_dev == nullptr ||
+      y_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear: null pointer%s");
+  if (!aligned16(a_codes_dev) || !aligned16(a_scales_dev) || !aligned16(w_codes_dev) ||
+      !aligned16(w_scales_dev) || !aligned16(y_dev) || (bias_dev != nullptr && !aligned16(bias_dev)))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear: every pointer must be 16-byte aligned%s");
+  if (int st = check_device()) return st;
+  const char* why = nullptr;
+  cudaError_t e = fh::launch_nvfp4_linear(a_codes_dev, a_scales_dev, a_gscale, w_codes_dev, w_scales_dev,
+                                          w_gscale, bias_dev, y_dev, M, N, K, (cudaStream_t)stream, &why);
+  if (e == cudaErrorNotSupported && why != nullptr) return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear: %s", why);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear launch");
+}
+
+int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows, int64_t K,
+                          fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (rows < 0 || K <= 0 || K % 64 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_scales_to_rowmajor: need rows >= 0, K > 0, K %% 64 == 0%s");
+  if (rows == 0) return FH_OK;
+  if (tiled_dev == nullptr || rowmajor_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_scales_to_rowmajor: null pointer%s");
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_scales_to_rowmajor(tiled_dev, rowmajor_dev, rows, K, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_scales_to_rowmajor launch");
+}
+
+int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (n < 0) return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_gelu_bf16: n must be >= 0%s");
+  if (n == 0) return FH_OK;
+  if (x_dev == nullptr || y_dev == nullptr) return fail(FH_ERR_INVALID_ARG, "fh_gelu_bf16: null pointer%s");
+  if (!aligned16(x_dev) || !aligned16(y_dev))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_gelu_bf16: x and y must be 16-byte aligned%s");
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_gelu(x_dev, y_dev, n, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_gelu_bf16 launch");
+}
+
+int fh_device_status(fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (int st = check_device()) return st;
+  unsigned int bits = 0;
+  cudaError_t e = fh::read_and_clear_device_error(&bits, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fh_device_status");
+  if (bits & fh::kDevErrTimeout)
+    return fail(FH_ERR_TIMEOUT, "a kernel gave up on a bounded on-chip wait%s");
+  return FH_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,565 @@
+// fh_gemm.cu -- NVFP4 linear layer on the sm_100a tcgen05 tensor cores.
+//
+//   y[m, n] = bf16( alpha * sum_k A[m,k] W[n,k] + bias[n] ),  alpha = s_gA * s_gW
+//
+// with A, W NVFP4 (E2M1 codes, one E4M3 scale per 16 elements along K).  This
+// is the FP4 matmul that FastH3 runs on Blackwell tensor cores (FastH3 thread
+// digest, farwalk.ai, tweet 5/8; FastH3 Trim, comfyui-wiki news, "How fast it
+// runs": the RTX 4090 lacks FP4 tensor cores, Blackwell has them).
+//
+// Design (one CTA per SM, persistent over 128 x 192 output tiles):
+//   warp 0      TMA producer: per 256-wide K stage, a 128 x 128-byte A tile and
+//               a 192 x 128-byte W tile (128-byte swizzle) by tensor TMA, and
+//               the stage's scale atoms (512 bytes = 128 rows x 64 K) by bulk
+//               copies, all completing on the stage's mbarrier.
+//   warp 1      allocates TMEM (512 columns); one lane copies the stage's scale
+//               atoms from shared memory to TMEM (tcgen05.cp) and issues four
+//               tcgen05.mma kind::mxf4nvf4 block_scale (M=128, N=192, K=64) per
+//               stage into one of two TMEM accumulators; tcgen05.commit frees the
+//               stage and, after the last stage, hands the accumulator over.
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, alpha * acc + bias
+//               in FP32, BF16 round-to-nearest-even, 128-byte-swizzled staging
+//               in shared memory and TMA stores, while the MMA warp already fills
+//               the other accumulator.
+// TMEM columns: accumulators [0, 192) and [192, 384); A scales [384, 400)
+// (4 columns per K=64 step); W scales [400, 432) (8 columns per K=64 step:
+// two 128-row scale blocks, since a 192-row tile starts at row 0 or 64 of a
+// 128-row scale block; odd tiles read from column +2).
+// Every mbarrier wait is bounded; on expiry the kernel sets the device error
+// word, stops issuing work, drains what it issued and frees its TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fh_internal.h"
+
+namespace fh {
+
+namespace {
+
+__device__ unsigned int g_device_error = 0;
+
+constexpr int BM = 128;
+constexpr int BN = 192;
+constexpr int BK = 256;                  // FP4 elements per stage = 128 bytes per row
+constexpr int kMmaK = 64;                // K of one tcgen05.mma kind::mxf4nvf4
+constexpr int kKSteps = BK / kMmaK;      // 4
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK / 2;     // 16384
+constexpr int kBBytes = BN * BK / 2;     // 24576
+constexpr int kAtomBytes = 512;          // 128 rows x 4 scales
+constexpr int kSFABytes = kKSteps * kAtomBytes;      // 2048
+constexpr int kSFBBytes = 2 * kKSteps * kAtomBytes;  // 4096
+constexpr int kEpiWarps = 4;
+constexpr int kEpiCols = 64;                          // columns per TMA store box
+constexpr int kEpiBufBytes = 32 * kEpiCols * 2;       // 4096: 32 rows x 128 bytes
+constexpr int kThreads = 64 + 32 * kEpiWarps;         // 192
+constexpr int kTmemCols = 512;
+constexpr int kAccCols = BN;
+constexpr int kSfaCol = 2 * kAccCols;                 // 384
+constexpr int kSfbCol = kSfaCol + 4 * kKSteps;        // 400
+
+constexpr int kOffA = 0;
+constexpr int kOffB = kOffA + kStages * kABytes;
+constexpr int kOffSFA = kOffB + kStages * kBBytes;
+constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
+constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
+constexpr int kOffBar = kOffEpi + kEpiWarps * 2 * kEpiBufBytes;
+constexpr int kNumBars = 2 * kStages + 4 + 1;  // full, empty, acc full x2, acc empty x2, drain
+constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
+constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+
+static_assert(kOffB % 1024 == 0 && kOffSFA % 1024 == 0 && kOffEpi % 1024 == 0, "alignment");
+static_assert(kSmemAlloc <= 232448, "shared memory budget");
+static_assert(kSfbCol + 8 * kKSteps <= kTmemCols, "TMEM budget");
+
+// Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format
+// 1), both K-major, UE4M3 scales, N >> 3 at bit 17, M >> 4 at bit 24, dense,
+// K = 64, scale-factor ids 0.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+struct Params {
+  const uint8_t* sfa;
+  const uint8_t* sfb;
+  const uint16_t* bias;
+  float alpha;
+  int M, N, K;
+  int n_tiles, num_tiles, k_stages;
+  int ksteps_total;  // K / 64
+  int sf_katoms;     // K / 64: 512-byte atoms per 128-row scale block
+  int n_sf_blocks;   // ceil(N / 128)
+};
+
+// ---- PTX wrappers ------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for phase `parity` of an mbarrier.  Gives up after ~4 s (or
+// when another role of the CTA already gave up), setting the device error word
+// and the CTA's abort flag.
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1; i < (1u << 30); ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u) {
+      if (*abort) return false;
+      if (global_ns() - t0 > kWaitLimitNs) break;
+    }
+  }
+  atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+  *abort = 1;
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor, K-major.  swizzle128: 128-byte rows in
+// 1024-byte swizzle atoms (stride between 8-row groups 1024 bytes); otherwise
+// no swizzle with 16-byte rows (stride between 8-row groups 128 bytes).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, bool swizzle128) {
+  uint64_t d = (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;                            // leading byte offset (unused here)
+  d |= (uint64_t)((swizzle128 ? 1024u : 128u) >> 4) << 32;  // stride byte offset
+  d |= (uint64_t)1u << 46;                            // descriptor version (sm_100)
+  d |= (uint64_t)(swizzle128 ? 2u : 0u) << 61;        // layout type
+  return d;
+}
+
+__device__ __forceinline__ void tc_cp_32x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate,
+                                       uint32_t sfa_tmem, uint32_t sfb_tmem) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
+      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 32 consecutive TMEM columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld_32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ---- kernel ----------------------------------------------------------------
+
+__global__ void __launch_bounds__(kThreads, 1)
+    nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmY, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + kOffBar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(accf_bar(a), 1);
+      mbar_init(acce_bar(a), kEpiWarps);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmY)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ===================== TMA producer =====================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
+        const int m0 = m_tile * BM, n0 = n_tile * BN;
+        const int jb0 = n0 / 128;
+        for (int kt = 0; kt < p.k_stages; ++kt) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
+          const uint32_t sf_bytes = (uint32_t)ks * kAtomBytes;
+          const int nsfb = (jb0 + 1 < p.n_sf_blocks) ? 2 : 1;
+          const uint32_t fb = full_bar(stage);
+          mbar_arrive_expect_tx(fb, kABytes + kBBytes + sf_bytes * (1 + nsfb));
+          tma_load_2d(sbase + kOffA + stage * kABytes, &tmA, fb, kt * (BK / 2), m0);
+          tma_load_2d(sbase + kOffB + stage * kBBytes, &tmB, fb, kt * (BK / 2), n0);
+          const size_t katom0 = (size_t)kt * kKSteps;
+          bulk_load(sbase + kOffSFA + stage * kSFABytes,
+                    p.sfa + ((size_t)m_tile * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, fb);
+          for (int r = 0; r < nsfb; ++r)
+            bulk_load(sbase + kOffSFB + stage * kSFBBytes + r * (kKSteps * kAtomBytes),
+                      p.sfb + ((size_t)(jb0 + r) * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, fb);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Drain: wait until every load this thread issued has landed, so no
+      // copy still targets shared memory when the CTA retires.
+      for (int s = 0; s < kStages; ++s) {
+        // Stage s was last filled in the phase before `phase` if s >= stage.
+        const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+        wait_bounded(full_bar(s), par, abort_flag);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================== MMA issuer =====================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int n_tile = t % p.n_tiles;
+        const uint32_t sfb_shift = (uint32_t)((n_tile * BN) % 128) / 32u;  // 0 or 2
+        if (!wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
+        for (int kt = 0; kt < p.k_stages; ++kt) {
+          if (!wait_bounded(full_bar(stage), phase, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
+          const uint32_t a_addr = sbase + kOffA + stage * kABytes;
+          const uint32_t b_addr = sbase + kOffB + stage * kBBytes;
+          const uint32_t sfa_addr = sbase + kOffSFA + stage * kSFABytes;
+          const uint32_t sfb_addr = sbase + kOffSFB + stage * kSFBBytes;
+          for (int k = 0; k < ks; ++k) {
+            tc_cp_32x128b(tmem_base + kSfaCol + 4 * k, smem_desc(sfa_addr + k * kAtomBytes, false));
+            tc_cp_32x128b(tmem_base + kSfbCol + 8 * k, smem_desc(sfb_addr + k * kAtomBytes, false));
+            tc_cp_32x128b(tmem_base + kSfbCol + 8 * k + 4,
+                          smem_desc(sfb_addr + kKSteps * kAtomBytes + k * kAtomBytes, false));
+          }
+          for (int k = 0; k < ks; ++k) {
+            tc_mma(d_tmem, smem_desc(a_addr + k * (kMmaK / 2), true),
+                   smem_desc(b_addr + k * (kMmaK / 2), true), (kt | k) != 0 ? 1u : 0u,
+                   tmem_base + kSfaCol + 4 * k, tmem_base + kSfbCol + 8 * k + sfb_shift);
+          }
+          tc_commit(empty_bar(stage));  // frees the stage once these MMAs have read it
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(acc));  // accumulator ready for the epilogue
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      // Drain: every MMA issued above has completed before TMEM is released.
+      tc_commit(drain_bar);
+      wait_bounded(drain_bar, 0, abort_flag);
+    }
+  } else {
+    // ===================== epilogue =====================
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    uint8_t* stage_buf = smem + kOffEpi + (warp - 2) * 2 * kEpiBufBytes;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    int buf = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+      const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
+      const int m0 = m_tile * BM, n0 = n_tile * BN;
+      if (!wait_bounded(accf_bar(acc), acc_phase, abort_flag)) break;
+      tc_fence_after();
+      for (int c = 0; c < BN / kEpiCols; ++c) {
+        const int col0 = n0 + c * kEpiCols;
+        if (col0 >= p.N) break;  // warp-uniform
+        uint32_t v[2][32];
+        const uint32_t taddr = tmem_base + lane_base + (uint32_t)(acc * kAccCols + c * kEpiCols);
+        tmem_ld_32(taddr, v[0]);
+        tmem_ld_32(taddr + 32, v[1]);
+        tmem_ld_wait();
+        // Bias for these 64 columns (the same for every lane: broadcast loads).
+        float bv[kEpiCols];
+#pragma unroll
+        for (int i = 0; i < kEpiCols / 8; ++i) {
+          uint4 u = make_uint4(0, 0, 0, 0);
+          if (p.bias != nullptr && col0 + 8 * i < p.N)
+            u = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + 8 * i));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            bv[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
+            bv[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+          }
+        }
+        uint32_t packed[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int cc = 2 * j;
+          const float y0 = fmaf(p.alpha, __uint_as_float(v[cc >> 5][cc & 31]), bv[cc]);
+          const float y1 = fmaf(p.alpha, __uint_as_float(v[(cc + 1) >> 5][(cc + 1) & 31]), bv[cc + 1]);
+          packed[j] = pack_bf16x2(y0, y1);
+        }
+        // Reuse a staging buffer only after its previous TMA store has read it.
+        if (lane == 0) bulk_wait_read_1();
+        __syncwarp();
+        uint8_t* sb = stage_buf + buf * kEpiBufBytes;
+        const uint32_t row = (uint32_t)lane;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t chunk = (uint32_t)i ^ (row & 7u);  // 128-byte swizzle
+          *reinterpret_cast<uint4*>(sb + row * 128 + chunk * 16) =
+              make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && m0 + 32 * q < p.M) {  // rows past M: nothing to store
+          tma_store_2d(&tmY, smem_u32(sb), col0, m0 + 32 * q);
+        }
+        if (lane == 0) bulk_commit();
+        buf ^= 1;
+      }
+      // All TMEM reads of this accumulator are done: hand it back to the MMA warp.
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+  }
+}
+
+// ---- host side ----------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t read_and_clear_device_error(unsigned int* bits, cudaStream_t s) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof v);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+  *bits = v;
+  return e;
+}
+
+cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,
+                                const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
+                                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                                cudaStream_t s, const char** why) {
+  CUtensorMap tmA, tmB, tmY;
+  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M,
+                   (uint64_t)K / 2, BK / 2, BM) ||
+      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N,
+                   (uint64_t)K / 2, BK / 2, BN) ||
+      !make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
+                   (uint64_t)N * 2, kEpiCols, 32)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or a layout rule violated)";
+    return cudaErrorNotSupported;
+  }
+  Params p;
+  p.sfa = a_scales;
+  p.sfb = w_scales;
+  p.bias = bias;
+  p.alpha = a_g * w_g;
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  const int m_tiles = (int)((M + BM - 1) / BM);
+  p.n_tiles = (int)((N + BN - 1) / BN);
+  p.num_tiles = m_tiles * p.n_tiles;
+  p.k_stages = (int)((K + BK - 1) / BK);
+  p.ksteps_total = (int)(K / kMmaK);
+  p.sf_katoms = (int)(K / kMmaK);
+  p.n_sf_blocks = (int)((N + 127) / 128);
+
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(nvfp4_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
+  nvfp4_linear_kernel<<<grid, kThreads, kSmemAlloc, s>>>(tmA, tmB, tmY, p);
+  return cudaGetLastError();
+}
+
+}  // namespace fh

@@ -1,0 +1,41 @@
+// fh_internal.h -- declarations shared by the CUDA translation units of libfh.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fh.h"
+
+namespace fh {
+
+// Device error word bits (read and cleared by fh_device_status).
+enum : unsigned int {
+  kDevErrTimeout = 1u,  // a bounded mbarrier wait expired
+};
+
+// Host side: synchronize `s`, then read and clear the device error word of the
+// current device (fh_gemm.cu owns the word).
+cudaError_t read_and_clear_device_error(unsigned int* bits, cudaStream_t s);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Quantizer / calibration / glue launchers (fh_quant.cu).  Arguments are
+// validated by the caller.
+cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float sg,
+                            uint8_t* codes, uint8_t* scales, unsigned long long* clip,
+                            int layout, cudaStream_t s);
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, float* amax,
+                        cudaStream_t s);
+cudaError_t launch_scales_to_rowmajor(const uint8_t* tiled, uint8_t* rowmajor, int64_t rows,
+                                      int64_t K, cudaStream_t s);
+cudaError_t launch_gelu(const uint16_t* x, uint16_t* y, int64_t n, cudaStream_t s);
+
+// GEMM launcher (fh_gemm.cu).  Returns a CUDA error, or cudaErrorNotSupported
+// when the tensor maps cannot be built (message in *why).
+cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,
+                                const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
+                                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N,
+                                int64_t K, cudaStream_t s, const char** why);
+
+}  // namespace fh

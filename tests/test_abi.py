@@ -1,0 +1,116 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/fh.h declares, and its host-only logic (scale rule, buffer sizes,
+argument validation) behaves as documented.  No call here reaches a GPU."""
+import ctypes
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synthetic as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "fh_build", os.path.join(ROOT, "nvfp4_quantized_linear_fh_b200", "build.py"))
+    build = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(build)
+    path = build.build()
+    L = ctypes.CDLL(path)
+    L.fh_scale_from_amax.restype = ctypes.c_float
+    L.fh_scale_from_amax.argtypes = [ctypes.c_float]
+    L.fh_scales_bytes.restype = ctypes.c_size_t
+    L.fh_scales_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int]
+    L.fh_last_error.restype = ctypes.c_char_p
+    return L
+
+
+def declared_entry_points():
+    with open(os.path.join(ROOT, "include", "fh.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:int|float|size_t|const char\*)\s+(fh_\w+)\(", text, re.M)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_entry_points()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_binding_wraps_every_entry_point():
+    import nvfp4_quantized_linear_fh_b200 as fh
+    for n in declared_entry_points():
+        assert callable(getattr(fh, n)), n
+
+
+def test_scale_from_amax_matches_oracle(lib):
+    rng = np.random.default_rng(0)
+    vals = np.concatenate([[0.0, 2688.0, 1344.0, 1096.0, 4.5, 1e-30, 3e38],
+                           np.exp(rng.uniform(np.log(1e-8), np.log(1e8), 2000))]).astype(np.float32)
+    for a in vals:
+        assert lib.fh_scale_from_amax(float(a)) == oracle.scale_from_amax(float(a)), a
+    assert math.isnan(lib.fh_scale_from_amax(-1.0))
+    assert math.isnan(lib.fh_scale_from_amax(float("inf")))
+
+
+def test_scales_bytes(lib):
+    assert lib.fh_scales_bytes(100, 48, 0) == 300
+    assert lib.fh_scales_bytes(100, 64, 1) == 128 * 4
+    assert lib.fh_scales_bytes(129, 2688, 1) == oracle.tiled_scales_bytes(129, 2688) == 256 * 168
+    assert lib.fh_scales_bytes(10, 48, 1) == 0      # K % 64 != 0
+    assert lib.fh_scales_bytes(10, 20, 0) == 0      # K % 16 != 0
+    assert lib.fh_scales_bytes(10, 64, 7) == 0
+
+
+def test_argument_validation_without_gpu(lib):
+    """Malformed calls are rejected before any device work."""
+    P = ctypes.c_void_p
+    fake = P(16)
+    # fh_quantize_act(x, M, K, ldx, sg, codes, scales, clip, layout, stream)
+    q = lib.fh_quantize_act
+    q.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_float, P, P, P, ctypes.c_int, P]
+    assert q(fake, 4, 24, 24, 1.0, fake, fake, None, 0, None) == 2            # K % 16
+    assert q(fake, 4, 48, 48, 1.0, fake, fake, None, 1, None) == 2            # tiled needs K % 64
+    assert q(fake, 4, 64, 60, 1.0, fake, fake, None, 0, None) == 2            # ldx < K
+    assert q(fake, 4, 64, 64, 0.0, fake, fake, None, 0, None) == 1            # scale <= 0
+    assert q(fake, 4, 64, 64, float("nan"), fake, fake, None, 0, None) == 1
+    assert q(fake, 4, 64, 64, 1.0, fake, fake, None, 5, None) == 1            # layout
+    assert q(None, 4, 64, 64, 1.0, fake, fake, None, 0, None) == 1            # null x
+    assert q(P(18), 4, 64, 64, 1.0, fake, fake, None, 0, None) == 2          # misaligned
+    assert q(fake, 0, 64, 64, 1.0, fake, fake, None, 0, None) == 0            # empty: nothing to do
+    assert b"16-byte" in lib.fh_last_error() or lib.fh_last_error() == b""
+    g = lib.fh_nvfp4_linear
+    g.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, P, P, ctypes.c_int64, ctypes.c_int64,
+                  ctypes.c_int64, P]
+    assert g(fake, fake, 1.0, fake, fake, 1.0, None, fake, 128, 256, 96, None) == 2   # K % 64
+    assert g(fake, fake, 1.0, fake, fake, 1.0, None, fake, 128, 250, 128, None) == 2  # N % 8
+    assert g(fake, fake, -1.0, fake, fake, 1.0, None, fake, 128, 256, 128, None) == 1
+    assert g(None, fake, 1.0, fake, fake, 1.0, None, fake, 128, 256, 128, None) == 1
+    assert g(fake, fake, 1.0, fake, fake, 1.0, None, fake, 0, 256, 128, None) == 0    # empty
+    assert g(fake, fake, 1.0, fake, fake, 1.0, None, fake, 128, 0, 128, None) == 0
+    a = lib.fh_amax
+    a.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P]
+    assert a(fake, 3, 5, 4, fake, None) == 2
+    assert a(fake, 0, 5, 5, fake, None) == 0
+    assert a(fake, 3, 5, 5, None, None) == 1
+
+
+def test_package_refuses_to_import_without_library(tmp_path):
+    """The binding fails loudly (no CPU fallback) when libfh.so is absent."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.join(ROOT, "nvfp4_quantized_linear_fh_b200")
+    dst = tmp_path / "nvfp4_quantized_linear_fh_b200"
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__", "csrc"))
+    r = subprocess.run([sys.executable, "-c", "import nvfp4_quantized_linear_fh_b200"], cwd=tmp_path,
+                       capture_output=True, text=True)
+    assert r.returncode != 0 and "no CPU fallback" in r.stderr

@@ -1,0 +1,140 @@
+"""GPU parity of the tcgen05 NVFP4 linear layer against the oracle's binary64
+dequantized product: |y - y_ref| <= 2^-8 |y_ref| + 1e-5 sum_k |a_k w_k| per
+output (the oracle quantizes the same BF16 inputs itself; the quantizer's
+bit-exactness is checked on the same inputs first)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic as S
+from _gpu_util import check_linear, check_quantize, fh, quantize_tiled, sample_rows, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def run_layer(x_bits, w_bits, b_bits, sg_a, sg_w):
+    m = fh()
+    M, K = x_bits.shape
+    N = w_bits.shape[0]
+    ac, asc, aclip = quantize_tiled(to_dev(x_bits), sg_a)
+    wc, wsc, _ = quantize_tiled(to_dev(w_bits), sg_w)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    y.fill_(float("nan"))
+    bias = None if b_bits is None else to_dev(b_bits)
+    m.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, bias, y)
+    torch.cuda.synchronize()
+    return y, int(aclip.item())
+
+
+SMALL = [(1, 64, 8), (100, 128, 200), (128, 256, 256), (129, 192, 392), (300, 320, 192),
+         (257, 2688, 384), (64, 512, 64), (130, 1024, 136)]
+
+
+@pytest.mark.parametrize("M,K,N", SMALL)
+def test_small_and_ragged_shapes(M, K, N):
+    x = S.random_bf16(("lin", M, K, "x"), (M, K), 1.0)
+    w = S.random_bf16(("lin", M, K, "w"), (N, K), 0.02)
+    b = S.random_bf16(("lin", M, K, "b"), (N,), 0.01)
+    sg_a = oracle.scale_from_amax(oracle.amax(x))
+    sg_w = oracle.scale_from_amax(oracle.amax(w))
+    check_quantize(x, sg_a, 1)
+    check_quantize(w, sg_w, 1)
+    y, _ = run_layer(x, w, b, sg_a, sg_w)
+    check_linear(y, x, sg_a, w, sg_w, b)
+
+
+def test_no_bias_and_unit_scales():
+    M, K, N = 130, 256, 200
+    x = S.random_bf16(("lin", "nobias", "x"), (M, K), 2.0)
+    w = S.random_bf16(("lin", "nobias", "w"), (N, K), 2.0)
+    y, _ = run_layer(x, w, None, 1.0, 1.0)
+    check_linear(y, x, 1.0, w, 1.0, None)
+
+
+def test_tiny_workload():
+    layer = S.workloads()["tiny"][0]
+    calib = S.activation_batches(layer, 0, layer.n_calib)
+    sg_a = oracle.scale_from_amax(oracle.amax(calib))
+    x = S.activations(layer)
+    w, b = S.weights(layer), S.bias(layer)
+    sg_w = oracle.scale_from_amax(oracle.amax(w))
+    y, clips = run_layer(x, w, b, sg_a, sg_w)
+    assert clips == 0
+    check_linear(y, x, sg_a, w, sg_w, b)
+
+
+def layer_case(name, idx=0, calib_batches=None):
+    layer = S.workloads()[name][idx]
+    x = S.activations(layer)
+    n_cal = layer.n_calib if calib_batches is None else calib_batches
+    extra = S.activation_batches(layer, layer.n_eval_batches, n_cal - layer.n_eval_batches) \
+        if n_cal > layer.n_eval_batches else None
+    amax = max(oracle.amax(x), oracle.amax(extra) if extra is not None else 0.0)
+    w, b = S.weights(layer), S.bias(layer)
+    return layer, x, w, b, oracle.scale_from_amax(amax), oracle.scale_from_amax(oracle.amax(w))
+
+
+@pytest.mark.parametrize("name", ["attn_proj", "qkv"])
+def test_full_size_layer(name):
+    layer, x, w, b, sg_a, sg_w = layer_case(name)
+    y, clips = run_layer(x, w, b, sg_a, sg_w)
+    assert clips == 0
+    check_quantize(w, sg_w, 1)
+    rows = sample_rows(layer.M, 48)
+    check_linear(y, x, sg_a, w, sg_w, b, rows=rows)
+    assert not torch.isnan(y).any()
+
+
+def test_ffn_pair_with_gelu():
+    """Up-projection, GELU on BF16, re-quantization with the down layer's own
+    calibrated scale, down-projection; both quantizers clip nothing."""
+    m = fh()
+    up = S.workloads()["ffn"][0]
+    down = S.workloads()["ffn"][1]
+    _, x, w1, b1, sg_x, sg_w1 = layer_case("ffn", 0, calib_batches=up.n_eval_batches)
+    w2, b2 = S.weights(down), S.bias(down)
+    sg_w2 = oracle.scale_from_amax(oracle.amax(w2))
+    h, clips = run_layer(x, w1, b1, sg_x, sg_w1)
+    assert clips == 0
+    g = torch.empty_like(h)
+    m.fh_gelu_bf16(h, g)
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    m.fh_amax(g, amax)                         # the down layer's calibration over the same batches
+    torch.cuda.synchronize()
+    sg_h = m.fh_scale_from_amax(amax.item())
+    g_bits = g.view(torch.int16).cpu().numpy().view(np.uint16)
+    rows = sample_rows(up.M, 32, seed=3)
+    check_quantize(g_bits[rows], sg_h, 1)
+    y, clips2 = run_layer(g_bits, w2, b2, sg_h, sg_w2)
+    assert clips2 == 0
+    check_linear(y, g_bits, sg_h, w2, sg_w2, b2, rows=rows)
+
+
+def test_block_sweep_layers_sampled():
+    """Two blocks of the 42-block sweep (all four layer shapes), rows sampled."""
+    sweep = S.workloads()["block_sweep"]
+    for layer in sweep[0:4] + sweep[-4:]:
+        small = S.Layer(layer.name, 4096, layer.K, layer.N, layer.batch, 64,
+                        channel_lognormal=layer.channel_lognormal, key=layer.key)
+        x = S.activations(small)
+        w, b = S.weights(layer), S.bias(layer)
+        sg_a = oracle.scale_from_amax(oracle.amax(x))
+        sg_w = oracle.scale_from_amax(oracle.amax(w))
+        y, clips = run_layer(x, w, b, sg_a, sg_w)
+        assert clips == 0
+        check_linear(y, x, sg_a, w, sg_w, b, rows=sample_rows(small.M, 16))
+
+
+def test_back_to_back_calls_reuse_nothing():
+    """Two different problems in a row on one stream give the same answers as alone."""
+    x1 = S.random_bf16(("b2b", 1), (256, 512), 1.0)
+    w1 = S.random_bf16(("b2b", 2), (384, 512), 0.02)
+    x2 = S.random_bf16(("b2b", 3), (130, 256), 1.0)
+    w2 = S.random_bf16(("b2b", 4), (200, 256), 0.02)
+    ya, _ = run_layer(x1, w1, None, 0.01, 0.0001)
+    yb, _ = run_layer(x2, w2, None, 0.01, 0.0001)
+    ya2, _ = run_layer(x1, w1, None, 0.01, 0.0001)
+    assert torch.equal(ya.view(torch.int16), ya2.view(torch.int16))
+    check_linear(yb, x2, 0.01, w2, 0.0001, None)
+    fh().fh_device_status()
