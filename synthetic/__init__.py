@@ -49,7 +49,10 @@ def derive_seed(*keys) -> int:
     z = np.array([0x5EED5EED5EED5EED], dtype=np.uint64)
     with np.errstate(over="ignore"):
         for k in keys:
-            v = zlib.crc32(k.encode()) if isinstance(k, str) else int(k)
+            if isinstance(k, (tuple, list)):
+                v = derive_seed(*k)
+            else:
+                v = zlib.crc32(k.encode()) if isinstance(k, str) else int(k)
             z = _mix(z + np.uint64(v & 0xFFFFFFFFFFFFFFFF) * _GAMMA + _GAMMA)
     return int(z[0])
 
