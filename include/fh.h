@@ -139,8 +139,9 @@ int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, flo
 int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows,
                           int64_t K, fh_stream_t stream);
 
-/* Exact-erf GELU on BF16, y = bf16(x/2 * (1 + erf(x/sqrt 2))) computed in
- * FP32; the activation between the two linear layers of the FFN.  n >= 0;
+/* Exact-erf GELU on BF16, y = bf16(x/2 * (1 + erf(x/sqrt 2))), evaluated in
+ * FP32 as x/2 * erfc(-x/sqrt 2) (no cancellation for negative x); the
+ * activation between the two linear layers of the FFN.  n >= 0;
  * x_dev and y_dev 16-byte aligned; in-place (x_dev == y_dev) is allowed. */
 int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t stream);
 

@@ -12,21 +12,25 @@
 // How the exact rounding stays cheap.  The inputs are BF16, so every decision
 // "is |x| (or amax_b) on this side of the exact real threshold t * S * s_g" is
 // the same as an integer compare of |x|'s 15 magnitude bits with the smallest
-// BF16 at (or beyond) the threshold.  Each CTA first builds, from s_g in FP64
+// BF16 at (or beyond) the threshold.  For a given s_g the host builds, in FP64
 // (where t * S * s_g is exact), these BF16 decision thresholds for all 126
-// finite non-zero scale codes.  For the elements it then uses the hardware
-// converter on x * (1 / (S s_g)) -- one multiply per element, two elements per
-// cvt -- but only for scale codes where it has checked, at every decision
-// boundary, that the converter's answer equals the exact one; the converter
-// and the multiply are monotone, so agreement at both sides of every boundary
+// finite non-zero scale codes, once per distinct s_g (cached), and passes them
+// to the kernel as a parameter; each CTA copies the 2.8 KB table to shared
+// memory.  Elements then go through the hardware converter on x * (1/(S s_g))
+// -- one multiply per element, two elements per cvt -- but only for scale
+// codes where the host has checked, at both sides of every decision boundary,
+// that the converter's documented rounding (round to nearest even, saturating
+// to the largest finite value) of that FP32 product gives the exact code; the
+// multiply and the converter are monotone, so agreement at every boundary
 // means agreement on every BF16 input.  Blocks whose scale code failed the
 // check (exact ties at non-power-of-two scales, typically) take the exact
-// threshold-compare path instead.  The block scale itself takes a converter
-// candidate and corrects it against the exact scale thresholds.
+// threshold-compare path.  The block scale takes a converter candidate and
+// corrects it against the exact scale thresholds.
 //
-// Memory: one thread owns one 16-element block per step: one 32-byte load,
-// one 8-byte code store, and one 4-byte store of four consecutive block scales
-// per four lanes (gathered with shuffles).  HBM-bound: 2.5625 bytes/element.
+// Memory: each thread owns two 16-element blocks per step: two 32-byte loads,
+// two 8-byte code stores, and one 4-byte store of four consecutive block
+// scales per four lanes (gathered with shuffles).  HBM-bound: 2.5625 bytes per
+// element.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -41,26 +45,143 @@ namespace {
 constexpr int kQuantThreads = 256;
 constexpr uint32_t kBf16Inf = 0x7F80u;
 
-// Exact positive E4M3 value of code c (1..126) in FP64.
-__device__ __forceinline__ double e4m3_magnitude(int c) {
+struct __align__(16) QuantTable {
+  uint16_t code_thr[128][8];  // [c][j<7]: smallest |x| (BF16 bits) whose exact magnitude code is >= j+1 at scale code c
+  uint16_t scale_thr[128];    // [c]: smallest block amax (BF16 bits) whose exact scale code is >= c
+  float inv[128];             // 1 / (S_c * s_g): multiplier of the converter path (0 for c == 0)
+  uint32_t fast_ok[4];        // bit c: the converter path is exact at scale code c
+};
+static_assert(sizeof(QuantTable) % 16 == 0, "table copy granularity");
+
+struct QuantParams {
+  QuantTable tab;
+  const uint16_t* x;
+  uint8_t* codes;
+  uint8_t* scales;
+  unsigned long long* clip;
+  int64_t M, K, ldx;
+  float inv6sg;       // 1 / (6 s_g): scale-code candidate multiplier
+  uint32_t clip_thr;  // smallest BF16 magnitude strictly beyond 2688 s_g
+  int wide;           // 32-byte loads allowed
+};
+
+// ---- host: the exact decision table for one global scale ----------------------
+
+// Exact positive E4M3 value of code c (1..126).
+double e4m3_magnitude(int c) {
   const int e = c >> 3, m = c & 7;
-  if (e == 0) return (double)m * 0x1p-9;
-  // (8 + m) * 2^(e - 10), with the power of two built exactly.
-  const double p2 = __longlong_as_double((long long)(1023 + e - 10) << 52);
-  return (double)(8 + m) * p2;
+  return e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
 }
 
-// Smallest BF16 (as 16 magnitude bits) that is >= T (strict == false) or > T
-// (strict == true), for T > 0; +Inf bits when no finite BF16 qualifies.
-__device__ uint32_t bf16_threshold(double T, bool strict) {
-  const float f = __double2float_ru(T);  // smallest FP32 >= T
-  const uint32_t u = __float_as_uint(f);
+// Smallest BF16 (16 magnitude bits) >= T, or > T when strict, for T > 0;
+// +Inf bits when no finite BF16 qualifies.
+uint32_t bf16_threshold(double T, bool strict) {
+  float f = (float)T;
+  if ((double)f < T) f = nextafterf(f, INFINITY);  // smallest FP32 >= T
+  uint32_t u;
+  memcpy(&u, &f, 4);
   uint32_t r = (u > 0x7F7F0000u) ? 0x7F800000u : ((u + 0xFFFFu) & 0xFFFF0000u);
-  if (strict && r != 0x7F800000u && (double)__uint_as_float(r) == T) r += 0x10000u;
+  if (strict && r != 0x7F800000u) {
+    float rf;
+    memcpy(&rf, &r, 4);
+    if ((double)rf == T) r += 0x10000u;
+  }
   return r >> 16;
 }
 
-// E4M3 x2 conversion (round to nearest even, saturating); returns the low byte's code.
+float bf16_bits_value(uint32_t bits16) {
+  const uint32_t u = bits16 << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+// The converter's documented result on a magnitude y >= 0: nearest E2M1 grid
+// point, ties to the even code, saturating at 6 (Inf included).
+uint32_t converter_e2m1(float y) {
+  static const float grid[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+  if (!(y < 6.0f)) return 7;
+  uint32_t c = 0;
+  for (int k = 1; k < 8; ++k) {
+    const float mid = 0.5f * (grid[k - 1] + grid[k]);
+    if (y > mid || (y == mid && (k & 1) == 0)) c = (uint32_t)k;
+  }
+  return c;
+}
+
+void build_table(float sg_f, QuantTable* t) {
+  const double sg = (double)sg_f;
+  static const double e2m1_mid[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
+  memset(t, 0, sizeof *t);
+  for (int c = 0; c < 128; ++c) {
+    // Block scale: codes c-1 and c meet at their midpoint; a tie goes to the even code.
+    if (c == 0) {
+      t->scale_thr[c] = 0;
+    } else if (c == 127) {
+      t->scale_thr[c] = (uint16_t)kBf16Inf;  // NaN code: never chosen
+    } else {
+      const double lo = (c == 1) ? 0.0 : e4m3_magnitude(c - 1);
+      const double mid = 0.5 * (lo + e4m3_magnitude(c));
+      t->scale_thr[c] = (uint16_t)bf16_threshold(mid * 6.0 * sg, ((c - 1) & 1) == 0);
+    }
+    // Element codes at scale code c: magnitude codes j and j+1 meet at the grid
+    // midpoint times S_c * s_g; a tie goes to the even code.
+    for (int j = 0; j < 8; ++j) {
+      uint32_t v = kBf16Inf;
+      if (j < 7 && c != 0 && c != 127)
+        v = bf16_threshold(e2m1_mid[j] * e4m3_magnitude(c) * sg, (j & 1) == 0);
+      t->code_thr[c][j] = (uint16_t)v;
+    }
+    t->inv[c] = (c == 0 || c == 127) ? 0.0f : (float)(1.0 / (e4m3_magnitude(c) * sg));
+  }
+  // Converter path check at both sides of every boundary and at the ends of the
+  // BF16 range.  Negative inputs give the same magnitude with the sign bit set.
+  for (int c = 0; c < 127; ++c) {
+    bool ok = true;
+    auto exact_mag = [&](uint32_t a) {
+      uint32_t m = 0;
+      for (int j = 0; j < 7; ++j) m += (a >= t->code_thr[c][j]) ? 1u : 0u;
+      return m;
+    };
+    auto probe = [&](uint32_t a) {
+      const float y = bf16_bits_value(a) * t->inv[c];  // the kernel's FP32 multiply
+      ok = ok && converter_e2m1(y) == exact_mag(a);
+    };
+    probe(0);
+    probe(0x7F7Fu);
+    for (int j = 0; j < 7; ++j) {
+      const uint32_t thr = t->code_thr[c][j];
+      if (thr <= 0x7F7Fu) {
+        probe(thr);
+        if (thr > 0) probe(thr - 1);
+      }
+    }
+    if (ok) t->fast_ok[c >> 5] |= 1u << (c & 31);
+  }
+}
+
+// Small per-thread cache: calibrated layers reuse one s_g for every call.
+const QuantTable& table_for(float sg) {
+  struct Entry {
+    float sg;
+    bool valid;
+    QuantTable t;
+  };
+  thread_local Entry cache[4] = {};
+  thread_local int next = 0;
+  for (auto& e : cache)
+    if (e.valid && e.sg == sg) return e.t;
+  Entry& e = cache[next];
+  next = (next + 1) & 3;
+  build_table(sg, &e.t);
+  e.sg = sg;
+  e.valid = true;
+  return e.t;
+}
+
+// ---- device --------------------------------------------------------------------
+
+// E4M3 x2 conversion (round to nearest even, saturating); the low byte's code.
 __device__ __forceinline__ uint32_t cvt_e4m3_sat(float v) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
@@ -76,96 +197,23 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
   return r;
 }
 
+// max(|a|, |b|) per BF16 half (sign bits = xor of the inputs' signs).
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 __device__ __forceinline__ float bf16_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
 
-// Fast-path code of one BF16 element at multiplier inv (4 bits with sign).
-__device__ __forceinline__ uint32_t fast_code(uint32_t bits16, float inv) {
-  return cvt_e2m1x2(0.0f, bf16_to_float(bits16) * inv) & 0xFu;
-}
-
-struct QuantTable {
-  uint16_t scale_thr[128];    // [c]: smallest |amax| (BF16 bits) whose exact scale code is >= c
-  uint16_t code_thr[128][8];  // [c][j<7]: smallest |x| whose exact magnitude code is >= j+1 at scale code c
-  float inv[128];             // 1 / (S_c * s_g) for the converter path (0 for c == 0)
-  uint32_t fast_ok[4];        // bit c: converter path verified exact at scale code c
-};
-
-// Exact magnitude code of |x| bits a at scale code c, from the table.
-__device__ __forceinline__ uint32_t exact_mag(const QuantTable& t, int c, uint32_t a) {
-  uint32_t m = 0;
-#pragma unroll
-  for (int j = 0; j < 7; ++j) m += (a >= t.code_thr[c][j]) ? 1u : 0u;
-  return m;
-}
-
-__device__ void build_table(QuantTable& t, float sg_f) {
-  const double sg = (double)sg_f;
-  const double e2m1_mid[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
-  for (int i = threadIdx.x; i < 128 * 8; i += blockDim.x) {
-    const int c = i >> 3, j = i & 7;
-    if (j == 7) {
-      uint32_t v;
-      if (c == 0) {
-        v = 0;
-      } else if (c == 127) {
-        v = kBf16Inf;  // sentinel: no amax reaches code 127 (NaN)
-      } else {
-        // Between codes c-1 and c; a tie goes to the even one.
-        const double lo = (c == 1) ? 0.0 : e4m3_magnitude(c - 1);
-        const double mid = 0.5 * (lo + e4m3_magnitude(c));
-        v = bf16_threshold(mid * 6.0 * sg, ((c - 1) & 1) == 0);
-      }
-      t.scale_thr[c] = (uint16_t)v;
-      t.code_thr[c][7] = (uint16_t)kBf16Inf;
-    } else {
-      uint32_t v = kBf16Inf;
-      if (c != 0 && c != 127) {
-        // Between magnitude codes j and j+1; a tie goes to the even one.
-        v = bf16_threshold(e2m1_mid[j] * e4m3_magnitude(c) * sg, (j & 1) == 0);
-      }
-      t.code_thr[c][j] = (uint16_t)v;
-    }
-  }
-  for (int c = threadIdx.x; c < 128; c += blockDim.x)
-    t.inv[c] = (c == 0 || c == 127) ? 0.0f : (float)(1.0 / (e4m3_magnitude(c) * sg));
-  if (threadIdx.x < 4) t.fast_ok[threadIdx.x] = (threadIdx.x == 3) ? 0x7FFFFFFFu : 0xFFFFFFFFu;
-  __syncthreads();
-
-  // Check the converter against the exact codes at both sides of every
-  // decision boundary, at the ends of the BF16 range, and for both signs.
-  for (int i = threadIdx.x; i < 127 * 8; i += blockDim.x) {
-    const int c = i >> 3, j = i & 7;
-    const float inv = t.inv[c];
-    uint32_t probe[2];
-    int np = 0;
-    if (j < 7) {
-      const uint32_t thr = t.code_thr[c][j];
-      if (thr <= 0x7F7Fu) {
-        probe[np++] = thr;
-        if (thr > 0) probe[np++] = thr - 1;
-      }
-    } else {
-      probe[np++] = 0;
-      probe[np++] = 0x7F7Fu;
-    }
-    bool ok = true;
-    for (int p = 0; p < np; ++p) {
-      const uint32_t a = probe[p];
-      const uint32_t want = exact_mag(t, c, a);
-      ok = ok && (fast_code(a, inv) == want) && (fast_code(a | 0x8000u, inv) == (want | 8u));
-    }
-    if (!ok) atomicAnd(&t.fast_ok[c >> 5], ~(1u << (c & 31)));
-  }
-  __syncthreads();
-}
-
-// 16 BF16 values (8 words) -> 8 code bytes (2 words), exact-threshold path.
-__device__ __forceinline__ void codes_exact(const QuantTable& t, int c, const uint32_t w[8],
-                                            uint32_t out[2]) {
+// 16 BF16 values (words w0..w7 in q0, q1) -> 8 code bytes, exact-threshold path.
+// Out of line: only blocks whose scale code failed the converter check get here.
+__device__ __noinline__ uint2 codes_exact(const QuantTable& t, uint32_t c, uint4 q0, uint4 q1) {
+  const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
   uint32_t thr[7];
 #pragma unroll
   for (int j = 0; j < 7; ++j) thr[j] = t.code_thr[c][j];
-  out[0] = out[1] = 0;
+  uint32_t out[2] = {0, 0};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint32_t lo = w[i] & 0xFFFFu, hi = w[i] >> 16;
@@ -178,22 +226,20 @@ __device__ __forceinline__ void codes_exact(const QuantTable& t, int c, const ui
     const uint32_t byte = (ml | ((lo >> 12) & 8u)) | ((mh | ((hi >> 12) & 8u)) << 4);
     out[i >> 2] |= byte << (8 * (i & 3));
   }
+  return make_uint2(out[0], out[1]);
 }
 
 // 16 BF16 values -> 8 code bytes via the converter at multiplier inv.
-__device__ __forceinline__ void codes_fast(float inv, const uint32_t w[8], uint32_t out[2]) {
+__device__ __forceinline__ void codes_fast(float inv, const uint32_t* w, uint32_t* out) {
   uint32_t b[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float lo = __uint_as_float(w[i] << 16) * inv;
-    const float hi = __uint_as_float(w[i] & 0xFFFF0000u) * inv;
-    b[i] = cvt_e2m1x2(hi, lo);
-  }
+  for (int i = 0; i < 8; ++i)
+    b[i] = cvt_e2m1x2(__uint_as_float(w[i] & 0xFFFF0000u) * inv, __uint_as_float(w[i] << 16) * inv);
   out[0] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
   out[1] = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
 }
 
-__device__ __forceinline__ void load_block(const uint16_t* p, uint32_t w[8], bool wide) {
+__device__ __forceinline__ void load_block(const uint16_t* p, uint32_t* w, bool wide) {
   if (wide) {
     asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
@@ -213,97 +259,110 @@ __device__ __forceinline__ int64_t tiled_offset(int64_t m, int64_t s, int64_t ka
   return ((m >> 7) * katoms + (s >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (s & 3);
 }
 
+// Quantize one loaded block of row m: stores its 8 code bytes, returns its
+// scale code and adds its clipped elements to clips.
+__device__ __forceinline__ uint32_t quantize_block(const QuantTable& tab, const QuantParams& p,
+                                                   const uint32_t* w, int64_t m, int64_t s,
+                                                   unsigned long long& clips) {
+  // Block amax over the magnitudes (a max, so exact).
+  const uint32_t r01 = max_abs_bf16x2(w[0], w[1]), r23 = max_abs_bf16x2(w[2], w[3]);
+  const uint32_t r45 = max_abs_bf16x2(w[4], w[5]), r67 = max_abs_bf16x2(w[6], w[7]);
+  const uint32_t r = max_abs_bf16x2(max_abs_bf16x2(r01, r23), max_abs_bf16x2(r45, r67));
+  const uint32_t amax = max_abs_bf16x2(r, __byte_perm(r, 0, 0x1032)) & 0x7FFFu;
+  // Scale code: converter candidate, corrected against the exact thresholds.
+  const float amax_f = bf16_to_float(amax);
+  uint32_t c = min(cvt_e4m3_sat(amax_f * p.inv6sg), 126u);
+  while (c < 126u && amax >= tab.scale_thr[c + 1]) ++c;
+  while (c > 0u && amax < tab.scale_thr[c]) --c;
+  uint2 out;
+  const float inv = tab.inv[c];
+  if (((tab.fast_ok[c >> 5] >> (c & 31)) & 1u) && (amax_f * inv <= 3.0e38f)) {
+    uint32_t o[2];
+    codes_fast(inv, w, o);
+    out = make_uint2(o[0], o[1]);
+  } else {
+    out = codes_exact(tab, c, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
+  }
+  *reinterpret_cast<uint2*>(p.codes + m * (p.K >> 1) + 8 * s) = out;
+  if (amax >= p.clip_thr) {  // only blocks reaching beyond the limit hold clipped elements
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      clips += ((w[i] & 0x7FFFu) >= p.clip_thr) ? 1u : 0u;
+      clips += (((w[i] >> 16) & 0x7FFFu) >= p.clip_thr) ? 1u : 0u;
+    }
+  }
+  return c;
+}
+
+template <bool kTiled, bool kGather4>
+__device__ __forceinline__ void store_scale(const QuantParams& p, uint32_t sc, bool valid, int lane, int64_t m,
+                                            int64_t s, int64_t nb, int64_t katoms) {
+  if (kGather4) {
+    // Lanes 4i..4i+3 hold four consecutive scales of one row.
+    const uint32_t pair = sc | (__shfl_down_sync(0xFFFFFFFFu, sc, 1) << 8);
+    const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
+    if (valid && (lane & 3) == 0)
+      *reinterpret_cast<uint32_t*>(p.scales + (kTiled ? tiled_offset(m, s, katoms) : m * nb + s)) = word;
+  } else if (valid) {
+    p.scales[kTiled ? tiled_offset(m, s, katoms) : m * nb + s] = (uint8_t)sc;
+  }
+}
+
 // kGather4: K/16 % 4 == 0, so lanes 4i..4i+3 own four consecutive scales of
 // one row and store them as one word.
 template <bool kTiled, bool kGather4>
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(
-    const uint16_t* __restrict__ x, int64_t M, int64_t K, int64_t ldx, float sg, float inv6sg,
-    uint32_t clip_thr, bool wide, uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    unsigned long long* __restrict__ clip_count) {
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p) {
   __shared__ QuantTable tab;
   __shared__ unsigned long long cta_clips;
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(&p.tab);
+    uint4* dst = reinterpret_cast<uint4*>(&tab);
+    for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 16); i += blockDim.x) dst[i] = src[i];
+  }
   if (threadIdx.x == 0) cta_clips = 0;
-  build_table(tab, sg);
+  __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const int64_t nb = K >> 4;
-  const int64_t total = M * nb;
+  const int64_t nb = p.K >> 4;
+  const int64_t total = p.M * nb;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t katoms = nb >> 2;
-  const int64_t dm = stride / nb, ds = stride % nb;
+  const int64_t dm = (2 * stride) / nb, ds = (2 * stride) % nb;
   int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  int64_t b = base + lane;
-  int64_t m = b / nb, s = b % nb;
+  // (m0, s0): this lane's first block of the step; (m1, s1): the second, one stride later.
+  int64_t m0 = (base + lane) / nb, s0 = (base + lane) % nb;
+  int64_t m1 = (base + stride + lane) / nb, s1 = (base + stride + lane) % nb;
   unsigned long long clips = 0;
 
-  for (; base < total; base += stride) {
-    const bool valid = b < total;
-    uint32_t w[8];
-    uint32_t sc = 0;
-    if (valid) {
-      load_block(x + m * ldx + 16 * s, w, wide);
-      // Block amax over the 15 magnitude bits of each BF16.
-      uint32_t mx = 0;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        uint32_t r;
-        asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(mx), "r"(w[i] & 0x7FFF7FFFu));
-        mx = r;
-      }
-      const uint32_t amax = max(mx & 0xFFFFu, mx >> 16);
-      // Scale code: converter candidate, corrected against the exact thresholds.
-      const float amax_f = bf16_to_float(amax);
-      uint32_t c = min(cvt_e4m3_sat(amax_f * inv6sg), 126u);
-      while (c < 126u && amax >= tab.scale_thr[c + 1]) ++c;
-      while (c > 0u && amax < tab.scale_thr[c]) --c;
-      sc = c;
-      // Element codes.
-      uint32_t out[2];
-      const float inv = tab.inv[c];
-      const bool fast = ((tab.fast_ok[c >> 5] >> (c & 31)) & 1u) && (amax_f * inv <= 3.0e38f);
-      if (fast)
-        codes_fast(inv, w, out);
-      else
-        codes_exact(tab, (int)c, w, out);
-      *reinterpret_cast<uint2*>(codes + m * (K >> 1) + 8 * s) = make_uint2(out[0], out[1]);
-      // Clipped elements: only blocks whose amax is beyond the limit have any.
-      if (amax >= clip_thr) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          clips += ((w[i] & 0x7FFFu) >= clip_thr) ? 1u : 0u;
-          clips += (((w[i] >> 16) & 0x7FFFu) >= clip_thr) ? 1u : 0u;
-        }
-      }
+  for (; base < total; base += 2 * stride) {
+    const bool v0 = base + lane < total, v1 = base + stride + lane < total;
+    uint32_t w0[8], w1[8];
+    if (v0) load_block(p.x + m0 * p.ldx + 16 * s0, w0, p.wide);
+    if (v1) load_block(p.x + m1 * p.ldx + 16 * s1, w1, p.wide);
+    const uint32_t sc0 = v0 ? quantize_block(tab, p, w0, m0, s0, clips) : 0u;
+    const uint32_t sc1 = v1 ? quantize_block(tab, p, w1, m1, s1, clips) : 0u;
+    store_scale<kTiled, kGather4>(p, sc0, v0, lane, m0, s0, nb, katoms);
+    store_scale<kTiled, kGather4>(p, sc1, v1, lane, m1, s1, nb, katoms);
+    s0 += ds;
+    m0 += dm;
+    if (s0 >= nb) {
+      s0 -= nb;
+      ++m0;
     }
-    if (kGather4) {
-      const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sc, 1);
-      const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sc, 2);
-      const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sc, 3);
-      if (valid && (lane & 3) == 0) {
-        const uint32_t word = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
-        const int64_t off = kTiled ? tiled_offset(m, s, katoms) : m * nb + s;
-        *reinterpret_cast<uint32_t*>(scales + off) = word;
-      }
-    } else if (valid) {
-      scales[kTiled ? tiled_offset(m, s, katoms) : m * nb + s] = (uint8_t)sc;
-    }
-    b += stride;
-    s += ds;
-    m += dm;
-    if (s >= nb) {
-      s -= nb;
-      ++m;
+    s1 += ds;
+    m1 += dm;
+    if (s1 >= nb) {
+      s1 -= nb;
+      ++m1;
     }
   }
 
   if (kTiled) {
     // Zero the scales of the padding rows M .. ceil(M/128)*128 - 1.
-    const int64_t mpad = ((M + 127) >> 7) << 7;
-    const int64_t npad = (mpad - M) * nb;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += stride) {
-      const int64_t pm = M + i / nb, ps = i % nb;
-      scales[tiled_offset(pm, ps, katoms)] = 0;
-    }
+    const int64_t mpad = ((p.M + 127) >> 7) << 7;
+    const int64_t npad = (mpad - p.M) * nb;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += stride)
+      p.scales[tiled_offset(p.M + i / nb, i % nb, katoms)] = 0;
   }
 
   // Clip count: warp sum, CTA sum, one atomic per CTA that saw any.
@@ -312,7 +371,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(
   for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xFFFFFFFFu, wsum, o);
   if (lane == 0 && wsum) atomicAdd(&cta_clips, wsum);
   __syncthreads();
-  if (threadIdx.x == 0 && cta_clips && clip_count) atomicAdd(clip_count, cta_clips);
+  if (threadIdx.x == 0 && cta_clips && p.clip) atomicAdd(p.clip, cta_clips);
 }
 
 // ---------------------------------------------------------------------------
@@ -377,7 +436,9 @@ __global__ void scales_to_rowmajor_kernel(const uint8_t* __restrict__ tiled,
 
 __device__ __forceinline__ uint32_t gelu_bits(uint32_t bits16) {
   const float v = bf16_to_float(bits16);
-  const float y = 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
+  // x/2 * erfc(-x/sqrt 2) == x/2 * (1 + erf(x/sqrt 2)), without the cancellation
+  // of 1 + erf for negative x.
+  const float y = 0.5f * v * erfcf(-v * 0.70710678118654752440f);
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y));
 }
 
@@ -406,46 +467,35 @@ int grid_for(int64_t work_items, int threads, int per_sm) {
 cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float sg,
                             uint8_t* codes, uint8_t* scales, unsigned long long* clip,
                             int layout, cudaStream_t s) {
+  QuantParams p;
+  memcpy(&p.tab, &table_for(sg), sizeof(QuantTable));
+  p.x = x;
+  p.codes = codes;
+  p.scales = scales;
+  p.clip = clip;
+  p.M = M;
+  p.K = K;
+  p.ldx = ldx;
+  p.inv6sg = (float)(1.0 / (6.0 * (double)sg));
+  p.wide = ((reinterpret_cast<uintptr_t>(x) & 31) == 0) && ((ldx % 16) == 0);
+  // Exact clip threshold: smallest BF16 magnitude strictly beyond 2688 * s_g
+  // (2688 * s_g is exact in FP64: 5 + 24 significant bits).
+  p.clip_thr = bf16_threshold(2688.0 * (double)sg, true);
   const int64_t nb = K / 16;
   const bool tiled = layout == FH_SCALES_MMA_TILED;
   const bool gather4 = (nb % 4) == 0;
-  const bool wide = ((reinterpret_cast<uintptr_t>(x) & 31) == 0) && ((ldx % 16) == 0);
-  // Exact clip threshold: smallest BF16 magnitude strictly beyond 2688 * s_g
-  // (2688 * s_g is exact in FP64: 5 + 24 significant bits).
-  const double limit = 2688.0 * (double)sg;
-  uint32_t clip_thr;
-  {
-    float f = (float)limit;
-    if ((double)f < limit) f = nextafterf(f, INFINITY);  // smallest FP32 >= limit
-    uint32_t u;
-    memcpy(&u, &f, 4);
-    if (u > 0x7F7F0000u) {
-      clip_thr = 0x7F80u;
-    } else {
-      uint32_t r = (u + 0xFFFFu) & 0xFFFF0000u;  // smallest BF16 >= limit
-      float rf;
-      memcpy(&rf, &r, 4);
-      if ((double)rf == limit) r += 0x10000u;  // strictly beyond
-      clip_thr = r >> 16;
-    }
-  }
-  const float inv6sg = (float)(1.0 / (6.0 * (double)sg));
   const int64_t mpad = tiled ? ((M + 127) / 128) * 128 : M;
-  const int grid = grid_for((mpad > M ? mpad : M) * nb, kQuantThreads, 8);
+  const int grid = grid_for((mpad * nb + 1) / 2, kQuantThreads, 4);
   if (tiled) {
     if (gather4)
-      quantize_kernel<true, true><<<grid, kQuantThreads, 0, s>>>(x, M, K, ldx, sg, inv6sg, clip_thr,
-                                                                 wide, codes, scales, clip);
+      quantize_kernel<true, true><<<grid, kQuantThreads, 0, s>>>(p);
     else
-      quantize_kernel<true, false><<<grid, kQuantThreads, 0, s>>>(x, M, K, ldx, sg, inv6sg, clip_thr,
-                                                                  wide, codes, scales, clip);
+      quantize_kernel<true, false><<<grid, kQuantThreads, 0, s>>>(p);
   } else {
     if (gather4)
-      quantize_kernel<false, true><<<grid, kQuantThreads, 0, s>>>(x, M, K, ldx, sg, inv6sg, clip_thr,
-                                                                  wide, codes, scales, clip);
+      quantize_kernel<false, true><<<grid, kQuantThreads, 0, s>>>(p);
     else
-      quantize_kernel<false, false><<<grid, kQuantThreads, 0, s>>>(x, M, K, ldx, sg, inv6sg,
-                                                                   clip_thr, wide, codes, scales, clip);
+      quantize_kernel<false, false><<<grid, kQuantThreads, 0, s>>>(p);
   }
   return cudaGetLastError();
 }
