@@ -250,10 +250,12 @@ void oracle_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,
   }
 }
 
-/* Exact-erf GELU in binary64: y = x/2 * (1 + erf(x / sqrt 2)). */
+/* Exact-erf GELU in binary64: y = x * Phi(x) = x/2 * (1 + erf(x / sqrt 2)),
+ * evaluated as x/2 * erfc(-x / sqrt 2), the same function written so that the
+ * negative tail (where 1 + erf cancels to 0) keeps its value. */
 void oracle_gelu(const uint16_t* x, int64_t n, double* y) {
   for (int64_t i = 0; i < n; ++i) {
     double v = oracle_bf16_value(x[i]);
-    y[i] = 0.5 * v * (1.0 + erf(v / sqrt(2.0)));
+    y[i] = 0.5 * v * erfc(-v / sqrt(2.0));
   }
 }

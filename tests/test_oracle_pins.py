@@ -355,7 +355,19 @@ def test_linear_one_hot(oracle_mod):
 
 
 def test_gelu(oracle_mod):
+    """GELU(x) = x Phi(x): tabulated normal CDF values, the identity
+    GELU(x) - GELU(-x) = x, and the asymptotic tail series
+    x Phi(x) ~ -phi(x) (1 - 1/x^2 + 3/x^4 - 15/x^6 + 105/x^8) for x -> -inf."""
     x = np.array([0x0000, 0x3F80, 0xBF80, 0x4000], np.uint16)   # 0, 1, -1, 2
     y = oracle_mod.gelu(x)
-    ref = [0.0, 0.8413447460685429, -0.15865525393145707, 1.9544997361036416]
+    ref = [0.0, 0.8413447460685429, -0.15865525393145707, 2 * 0.9772498680518208]
     np.testing.assert_allclose(y, ref, rtol=1e-15, atol=0)
+    v = S.random_bf16(("pin", "gelu"), (1000,), 3.0)
+    d = oracle_mod.gelu(v) - oracle_mod.gelu(v ^ np.uint16(0x8000))
+    np.testing.assert_allclose(d, S.bf16_to_f32(v).astype(np.float64), rtol=1e-14, atol=1e-300)
+    for xv in [-8.0, -9.0, -10.0, -12.0]:
+        series = 1 - 1 / xv**2 + 3 / xv**4 - 15 / xv**6 + 105 / xv**8
+        asym = -math.exp(-xv * xv / 2) / math.sqrt(2 * math.pi) * series
+        got = oracle_mod.gelu(S.to_bf16_bits(np.array([xv])))[0]
+        bound = 945 / xv**10 * 1.01     # the next term of the alternating series
+        assert abs(got - asym) <= abs(asym) * bound, (xv, got, asym)
