@@ -56,16 +56,29 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
+    def __init__(self, gpu_id: str):
+        self.gpu = gpu_id
         self.proc = None
-        self.lines = []
+        self.lines = []          # (host time, csv line)
+        self.t0 = self.t1 = None
+
+    def wait_first_sample(self, timeout: float = 3.0):
+        end = time.time() + timeout
+        while self.proc is not None and not self.lines and time.time() < end:
+            time.sleep(0.01)
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+        time.sleep(0.05)         # one more sample interval
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
@@ -74,7 +87,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -87,7 +100,11 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        # samples taken while the timed region ran (nvidia-smi reports each sample
+        # shortly after it is taken, so allow one interval of slack at the end)
+        lo, hi = (self.t0 or 0.0), (self.t1 or 1e30) + 0.04
+        window = [l for t, l in self.lines if lo <= t <= hi]
+        for line in window:
             parts = [x.strip() for x in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -102,7 +119,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "interval_ms": 20}
 
 
 def make_inputs(rank: int, M: int, quick: bool):
@@ -150,7 +167,6 @@ def bench_fh(args, rank, world, local_rank):
     ac, asc = fh.empty_quantized(M, K, device=dev)
     clip = torch.zeros(1, dtype=torch.int64, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)  # > L2 (126 MB)
     stream = torch.cuda.current_stream()
 
     def step():
@@ -168,14 +184,16 @@ def bench_fh(args, rank, world, local_rank):
     torch.cuda.synchronize()
     sampler = ClockSampler(f"GPU-{torch.cuda.get_device_properties(dev).uuid}")
     with sampler:
+        sampler.wait_first_sample()
+        sampler.mark_start()
         for i in range(args.steps):
-            flush.fill_(i)                      # evict the previous step's data from L2
             ev[i][0].record(stream)
             fh.fh_quantize_act(x, sg_a, ac, asc, clip)
             ev[i][1].record(stream)
             fh.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, bias, y)
             ev[i][2].record(stream)
         torch.cuda.synchronize()
+        sampler.mark_end()
     if world > 1:
         torch.distributed.barrier()
     t_quant = [ev[i][0].elapsed_time(ev[i][1]) * 1e-3 for i in range(args.steps)]
@@ -266,7 +284,8 @@ def main():
     pk = peaks()
     cfg = {"workload": f"fused QKV linear {args.M}x{WORKLOAD['K']}->{WORKLOAD['N']} (M x K -> N) per GPU",
            "M": args.M, "K": WORKLOAD["K"], "N": WORKLOAD["N"], "tokens_per_gpu": args.M,
-           "parallelism": f"dp{world} (token rows per GPU, replicas)", "l2": "flushed between steps (256 MB write)"}
+           "parallelism": f"dp{world} (token rows per GPU, replicas)",
+           "l2": "not flushed: each step's inputs and outputs exceed L2 (x 176 MB read, y 528 MB written)"}
 
     if args.impl == "reference":
         if rank != 0:
