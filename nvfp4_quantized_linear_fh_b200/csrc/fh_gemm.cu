@@ -7,24 +7,29 @@
 // digest, farwalk.ai, tweet 5/8; FastH3 Trim, comfyui-wiki news, "How fast it
 // runs": the RTX 4090 lacks FP4 tensor cores, Blackwell has them).
 //
-// Design (one CTA per SM, persistent over 128 x 192 output tiles):
+// Design (one CTA per SM, persistent over 128 x 192 output tiles, 320 threads):
 //   warp 0      TMA producer: per 256-wide K stage, a 128 x 128-byte A tile and
 //               a 192 x 128-byte W tile (128-byte swizzle) by tensor TMA, and
 //               the stage's scale atoms (512 bytes = 128 rows x 64 K) by bulk
 //               copies, all completing on the stage's mbarrier.
-//   warp 1      allocates TMEM (512 columns); one lane copies the stage's scale
-//               atoms from shared memory to TMEM (tcgen05.cp) and issues four
-//               tcgen05.mma kind::mxf4nvf4 block_scale (M=128, N=192, K=64) per
-//               stage into one of two TMEM accumulators; tcgen05.commit frees the
-//               stage and, after the last stage, hands the accumulator over.
+//   warp 1      allocates TMEM (512 columns); one lane issues four tcgen05.mma
+//               kind::mxf4nvf4 block_scale (M=128, N=192, K=64) per stage into
+//               one of two TMEM accumulators; tcgen05.commit frees the stage's
+//               shared memory and scale buffer and, after the last stage, hands
+//               the accumulator to the epilogue.
+//   warps 6..9  scale stagers, one per TMEM lane quadrant: copy the stage's
+//               scale atoms from shared memory into a 3-deep ring of TMEM scale
+//               buffers with tcgen05.st (each warp fills its own 32 lanes, which
+//               is the replication the MMA reads).  Moving the scales this way
+//               keeps them off the tensor pipe: tcgen05.cp of the same bytes
+//               serializes with the MMAs and would halve their rate.
 //   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, alpha * acc + bias
 //               in FP32, BF16 round-to-nearest-even, 128-byte-swizzled staging
 //               in shared memory and TMA stores, while the MMA warp already fills
 //               the other accumulator.
-// TMEM columns: accumulators [0, 192) and [192, 384); A scales [384, 400)
-// (4 columns per K=64 step); W scales [400, 432) (8 columns per K=64 step:
-// two 128-row scale blocks, since a 192-row tile starts at row 0 or 64 of a
-// 128-row scale block; odd tiles read from column +2).
+// TMEM columns: accumulators [0, 192) and [192, 384); three scale buffers of 40
+// columns from 384: per K=64 step, 4 columns of A scales (row r at lane r%32,
+// column r/32) then 6 columns of W scales for the tile's 192 rows.
 // Every mbarrier wait is bounded; on expiry the kernel sets the device error
 // word, stops issuing work, drains what it issued and frees its TMEM.
 #include <cuda.h>
@@ -52,27 +57,32 @@ constexpr int kAtomBytes = 512;          // 128 rows x 4 scales
 constexpr int kSFABytes = kKSteps * kAtomBytes;      // 2048
 constexpr int kSFBBytes = 2 * kKSteps * kAtomBytes;  // 4096
 constexpr int kEpiWarps = 4;
+constexpr int kSfWarps = 4;
 constexpr int kEpiCols = 64;                          // columns per TMA store box
 constexpr int kEpiBufBytes = 32 * kEpiCols * 2;       // 4096: 32 rows x 128 bytes
-constexpr int kThreads = 64 + 32 * kEpiWarps;         // 192
+constexpr int kThreads = 64 + 32 * (kEpiWarps + kSfWarps);  // 320
+constexpr int kFirstSfWarp = 2 + kEpiWarps;           // 6
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = BN;
-constexpr int kSfaCol = 2 * kAccCols;                 // 384
-constexpr int kSfbCol = kSfaCol + 4 * kKSteps;        // 400
+constexpr int kSfCols = 4 * kKSteps + 6 * kKSteps;    // 40 per stage: A 4, W 6 per K=64 step
+constexpr int kSfBufs = 3;
+constexpr int kSfCol0 = 2 * kAccCols;                 // 384
 
 constexpr int kOffA = 0;
 constexpr int kOffB = kOffA + kStages * kABytes;
 constexpr int kOffSFA = kOffB + kStages * kBBytes;
 constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
 constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
-constexpr int kOffBar = kOffEpi + kEpiWarps * 2 * kEpiBufBytes;
-constexpr int kNumBars = 2 * kStages + 4 + 1;  // full, empty, acc full x2, acc empty x2, drain
+constexpr int kOffBias = kOffEpi + kEpiWarps * 2 * kEpiBufBytes;
+constexpr int kOffBar = kOffBias + kEpiWarps * BN * 4;
+// full, empty (per stage); acc full, acc empty (x2); scale full, scale empty (x3); drain
+constexpr int kNumBars = 2 * kStages + 4 + 2 * kSfBufs + 1;
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
 constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
 
 static_assert(kOffB % 1024 == 0 && kOffSFA % 1024 == 0 && kOffEpi % 1024 == 0, "alignment");
 static_assert(kSmemAlloc <= 232448, "shared memory budget");
-static_assert(kSfbCol + 8 * kKSteps <= kTmemCols, "TMEM budget");
+static_assert(kSfCol0 + kSfBufs * kSfCols <= kTmemCols, "TMEM budget");
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format
 // 1), both K-major, UE4M3 scales, N >> 3 at bit 17, M >> 4 at bit 24, dense,
@@ -207,10 +217,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, bool swizzle128) {
   return d;
 }
 
-__device__ __forceinline__ void tc_cp_32x128b(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate,
                                        uint32_t sfa_tmem, uint32_t sfb_tmem) {
   asm volatile(
@@ -240,6 +246,32 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 16 / 8 consecutive TMEM columns of this thread's lane from registers.
+__device__ __forceinline__ void tmem_st_16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_8(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -247,6 +279,18 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // ---- kernel ----------------------------------------------------------------
+
+// Phase bookkeeping of a ring of `n` mbarrier-guarded slots.
+struct Ring {
+  int slot = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
 
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -260,7 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
   auto accf_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4);
+  auto sff_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 4 + b); };
+  auto sfe_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 4 + kSfBufs + b); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4 + 2 * kSfBufs);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 8);
 
@@ -275,6 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);
       mbar_init(acce_bar(a), kEpiWarps);
+    }
+    for (int b = 0; b < kSfBufs; ++b) {
+      mbar_init(sff_bar(b), kSfWarps);
+      mbar_init(sfe_bar(b), 1);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -297,86 +347,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ===================== TMA producer =====================
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring st;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
         const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
         const int m0 = m_tile * BM, n0 = n_tile * BN;
         const int jb0 = n0 / 128;
         for (int kt = 0; kt < p.k_stages; ++kt) {
-          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag)) {
+          if (!wait_bounded(empty_bar(st.slot), st.phase ^ 1u, abort_flag)) {
             ok = false;
             break;
           }
           const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
           const uint32_t sf_bytes = (uint32_t)ks * kAtomBytes;
           const int nsfb = (jb0 + 1 < p.n_sf_blocks) ? 2 : 1;
-          const uint32_t fb = full_bar(stage);
+          const uint32_t fb = full_bar(st.slot);
           mbar_arrive_expect_tx(fb, kABytes + kBBytes + sf_bytes * (1 + nsfb));
-          tma_load_2d(sbase + kOffA + stage * kABytes, &tmA, fb, kt * (BK / 2), m0);
-          tma_load_2d(sbase + kOffB + stage * kBBytes, &tmB, fb, kt * (BK / 2), n0);
+          tma_load_2d(sbase + kOffA + st.slot * kABytes, &tmA, fb, kt * (BK / 2), m0);
+          tma_load_2d(sbase + kOffB + st.slot * kBBytes, &tmB, fb, kt * (BK / 2), n0);
           const size_t katom0 = (size_t)kt * kKSteps;
-          bulk_load(sbase + kOffSFA + stage * kSFABytes,
+          bulk_load(sbase + kOffSFA + st.slot * kSFABytes,
                     p.sfa + ((size_t)m_tile * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, fb);
           for (int r = 0; r < nsfb; ++r)
-            bulk_load(sbase + kOffSFB + stage * kSFBBytes + r * (kKSteps * kAtomBytes),
+            bulk_load(sbase + kOffSFB + st.slot * kSFBBytes + r * (kKSteps * kAtomBytes),
                       p.sfb + ((size_t)(jb0 + r) * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, fb);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          st.next(kStages);
         }
       }
       // Drain: wait until every load this thread issued has landed, so no
       // copy still targets shared memory when the CTA retires.
       for (int s = 0; s < kStages; ++s) {
-        // Stage s was last filled in the phase before `phase` if s >= stage.
-        const uint32_t par = (s < stage) ? phase : (phase ^ 1u);
+        // Stage s was last filled in the phase before `phase` if s >= slot.
+        const uint32_t par = (s < st.slot) ? st.phase : (st.phase ^ 1u);
         wait_bounded(full_bar(s), par, abort_flag);
       }
     }
   } else if (warp == 1) {
     // ===================== MMA issuer =====================
     if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
+      Ring st, sf;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-        const int n_tile = t % p.n_tiles;
-        const uint32_t sfb_shift = (uint32_t)((n_tile * BN) % 128) / 32u;  // 0 or 2
         if (!wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
         for (int kt = 0; kt < p.k_stages; ++kt) {
-          if (!wait_bounded(full_bar(stage), phase, abort_flag)) {
+          if (!wait_bounded(full_bar(st.slot), st.phase, abort_flag) ||
+              !wait_bounded(sff_bar(sf.slot), sf.phase, abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
-          const uint32_t a_addr = sbase + kOffA + stage * kABytes;
-          const uint32_t b_addr = sbase + kOffB + stage * kBBytes;
-          const uint32_t sfa_addr = sbase + kOffSFA + stage * kSFABytes;
-          const uint32_t sfb_addr = sbase + kOffSFB + stage * kSFBBytes;
+          const uint32_t a_addr = sbase + kOffA + st.slot * kABytes;
+          const uint32_t b_addr = sbase + kOffB + st.slot * kBBytes;
+          const uint32_t sf_tmem = tmem_base + (uint32_t)(kSfCol0 + sf.slot * kSfCols);
           for (int k = 0; k < ks; ++k) {
-            tc_cp_32x128b(tmem_base + kSfaCol + 4 * k, smem_desc(sfa_addr + k * kAtomBytes, false));
-            tc_cp_32x128b(tmem_base + kSfbCol + 8 * k, smem_desc(sfb_addr + k * kAtomBytes, false));
-            tc_cp_32x128b(tmem_base + kSfbCol + 8 * k + 4,
-                          smem_desc(sfb_addr + kKSteps * kAtomBytes + k * kAtomBytes, false));
+            tc_mma(d_tmem, smem_desc(a_addr + k * (kMmaK / 2), true), smem_desc(b_addr + k * (kMmaK / 2), true),
+                   (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
           }
-          for (int k = 0; k < ks; ++k) {
-            tc_mma(d_tmem, smem_desc(a_addr + k * (kMmaK / 2), true),
-                   smem_desc(b_addr + k * (kMmaK / 2), true), (kt | k) != 0 ? 1u : 0u,
-                   tmem_base + kSfaCol + 4 * k, tmem_base + kSfbCol + 8 * k + sfb_shift);
-          }
-          tc_commit(empty_bar(stage));  // frees the stage once these MMAs have read it
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
+          tc_commit(empty_bar(st.slot));  // the stage's shared memory, once these MMAs have read it
+          tc_commit(sfe_bar(sf.slot));    // the scale buffer, likewise
+          st.next(kStages);
+          sf.next(kSfBufs);
         }
         if (!ok) break;
         tc_commit(accf_bar(acc));  // accumulator ready for the epilogue
@@ -389,17 +424,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_commit(drain_bar);
       wait_bounded(drain_bar, 0, abort_flag);
     }
+  } else if (warp >= kFirstSfWarp) {
+    // ===================== scale stagers =====================
+    // Lane l of the warp for quadrant q writes TMEM lane 32q + l.  A scale atom
+    // holds, at bytes 16 l .. 16 l + 15, the four K=64 scales of rows l, l+32,
+    // l+64, l+96: TMEM columns 0..3 of a K step (row r at column r/32).
+    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
+    Ring st, sf;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      const bool odd = ((t % p.n_tiles) * BN) % 128 != 0;  // tile starts at row 64 of a scale block
+      for (int kt = 0; kt < p.k_stages; ++kt) {
+        if (!wait_bounded(full_bar(st.slot), st.phase, abort_flag) ||
+            !wait_bounded(sfe_bar(sf.slot), sf.phase ^ 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sfa_addr = sbase + kOffSFA + st.slot * kSFABytes + lane * 16;
+        const uint32_t sfb_addr = sbase + kOffSFB + st.slot * kSFBBytes + lane * 16;
+        uint32_t va[16], vb[24];
+#pragma unroll
+        for (int k = 0; k < kKSteps; ++k) {
+          const uint4 a = lds128(sfa_addr + k * kAtomBytes);
+          va[4 * k] = a.x;
+          va[4 * k + 1] = a.y;
+          va[4 * k + 2] = a.z;
+          va[4 * k + 3] = a.w;
+          const uint4 b0 = lds128(sfb_addr + k * kAtomBytes);
+          const uint4 b1 = lds128(sfb_addr + kKSteps * kAtomBytes + k * kAtomBytes);
+          // The tile's 192 rows: rows 0..191 (even tile) or 64..255 (odd tile)
+          // of the two 128-row scale blocks, 32 rows per column.
+          vb[6 * k + 0] = odd ? b0.z : b0.x;
+          vb[6 * k + 1] = odd ? b0.w : b0.y;
+          vb[6 * k + 2] = odd ? b1.x : b0.z;
+          vb[6 * k + 3] = odd ? b1.y : b0.w;
+          vb[6 * k + 4] = odd ? b1.z : b1.x;
+          vb[6 * k + 5] = odd ? b1.w : b1.y;
+        }
+        const uint32_t col = tmem_base + lane_base + (uint32_t)(kSfCol0 + sf.slot * kSfCols);
+        uint32_t v16[16], v8[8];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v16[i] = va[i];
+        tmem_st_16(col, v16);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v16[i] = vb[i];
+        tmem_st_16(col + 16, v16);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v8[i] = vb[16 + i];
+        tmem_st_8(col + 32, v8);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sff_bar(sf.slot));
+        st.next(kStages);
+        sf.next(kSfBufs);
+      }
+    }
   } else {
     // ===================== epilogue =====================
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     uint8_t* stage_buf = smem + kOffEpi + (warp - 2) * 2 * kEpiBufBytes;
+    float* bias_s = reinterpret_cast<float*>(smem + kOffBias) + (warp - 2) * BN;
     int acc = 0;
     uint32_t acc_phase = 0;
     int buf = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
       const int m0 = m_tile * BM, n0 = n_tile * BN;
+      // The tile's bias, in FP32, staged in this warp's shared memory before
+      // the accumulator is ready (lanes 0..23 load 8 values each).
+      if (lane < BN / 8) {
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if (p.bias != nullptr && n0 + 8 * lane < p.N)
+          u = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * lane));
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        float4 f0 = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xFFFF0000u),
+                                __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xFFFF0000u));
+        float4 f1 = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xFFFF0000u),
+                                __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xFFFF0000u));
+        reinterpret_cast<float4*>(bias_s)[2 * lane] = f0;
+        reinterpret_cast<float4*>(bias_s)[2 * lane + 1] = f1;
+      }
+      __syncwarp();
       if (!wait_bounded(accf_bar(acc), acc_phase, abort_flag)) break;
       tc_fence_after();
       for (int c = 0; c < BN / kEpiCols; ++c) {
@@ -410,27 +518,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_32(taddr, v[0]);
         tmem_ld_32(taddr + 32, v[1]);
         tmem_ld_wait();
-        // Bias for these 64 columns (the same for every lane: broadcast loads).
-        float bv[kEpiCols];
-#pragma unroll
-        for (int i = 0; i < kEpiCols / 8; ++i) {
-          uint4 u = make_uint4(0, 0, 0, 0);
-          if (p.bias != nullptr && col0 + 8 * i < p.N)
-            u = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + 8 * i));
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            bv[8 * i + 2 * k] = __uint_as_float(w[k] << 16);
-            bv[8 * i + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-          }
-        }
         uint32_t packed[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int cc = 2 * j;
-          const float y0 = fmaf(p.alpha, __uint_as_float(v[cc >> 5][cc & 31]), bv[cc]);
-          const float y1 = fmaf(p.alpha, __uint_as_float(v[(cc + 1) >> 5][(cc + 1) & 31]), bv[cc + 1]);
-          packed[j] = pack_bf16x2(y0, y1);
+        for (int j = 0; j < 16; ++j) {
+          const float4 bv = reinterpret_cast<const float4*>(bias_s + c * kEpiCols)[j];
+          const int cc = 4 * j;
+          const float y0 = fmaf(p.alpha, __uint_as_float(v[cc >> 5][cc & 31]), bv.x);
+          const float y1 = fmaf(p.alpha, __uint_as_float(v[(cc + 1) >> 5][(cc + 1) & 31]), bv.y);
+          const float y2 = fmaf(p.alpha, __uint_as_float(v[(cc + 2) >> 5][(cc + 2) & 31]), bv.z);
+          const float y3 = fmaf(p.alpha, __uint_as_float(v[(cc + 3) >> 5][(cc + 3) & 31]), bv.w);
+          packed[2 * j] = pack_bf16x2(y0, y1);
+          packed[2 * j + 1] = pack_bf16x2(y2, y3);
         }
         // Reuse a staging buffer only after its previous TMA store has read it.
         if (lane == 0) bulk_wait_read_1();
