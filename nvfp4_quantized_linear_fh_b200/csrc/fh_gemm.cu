@@ -7,16 +7,23 @@
 // digest, farwalk.ai, tweet 5/8; FastH3 Trim, comfyui-wiki news, "How fast it
 // runs": the RTX 4090 lacks FP4 tensor cores, Blackwell has them).
 //
-// Design (one CTA per SM, persistent over 128 x 192 output tiles, 320 threads):
-//   warp 0      TMA producer: per 256-wide K stage, a 128 x 128-byte A tile and
-//               a 192 x 128-byte W tile (128-byte swizzle) by tensor TMA, and
-//               the stage's scale atoms (512 bytes = 128 rows x 64 K) by bulk
-//               copies, all completing on the stage's mbarrier.
-//   warp 1      allocates TMEM (512 columns); one lane issues four tcgen05.mma
-//               kind::mxf4nvf4 block_scale (M=128, N=192, K=64) per stage into
-//               one of two TMEM accumulators; tcgen05.commit frees the stage's
-//               shared memory and scale buffer and, after the last stage, hands
-//               the accumulator to the epilogue.
+// Design: persistent, warp-specialized, one CTA per SM.  By default two CTAs
+// of a cluster pair up on one 256 x 192 output tile with tcgen05.mma
+// cta_group::2 (each SM computes 128 rows; the 192 W rows are split 96/96
+// between the two SMs' shared memory, so each SM loads and holds half of W);
+// the single-CTA form (128 x 192 tiles) is the same code with kCta = 1.
+// Per CTA, 320 threads:
+//   warp 0      TMA producer: per 256-wide K stage, its 128 x 128-byte A tile
+//               and its (192 / kCta) x 128-byte W tile (128-byte swizzle) by
+//               tensor TMA completing on the leader CTA's stage barrier, and the
+//               stage's scale atoms (512 bytes = 128 rows x 64 K) by bulk copies
+//               completing on a barrier of its own CTA.
+//   warp 1      allocates TMEM (512 columns, both CTAs); in the leader CTA one
+//               lane issues four tcgen05.mma kind::mxf4nvf4 block_scale
+//               (M = 128 kCta, N = 192, K = 64) per stage into one of two TMEM
+//               accumulators; tcgen05.commit (multicast to the pair) frees the
+//               stage's shared memory and scale buffer and, after the last
+//               stage, hands the accumulator to both CTAs' epilogues.
 //   warps 6..9  scale stagers, one per TMEM lane quadrant: copy the stage's
 //               scale atoms from shared memory into a 3-deep ring of TMEM scale
 //               buffers with tcgen05.st (each warp fills its own 32 lanes, which
@@ -27,15 +34,17 @@
 //               in FP32, BF16 round-to-nearest-even, 128-byte-swizzled staging
 //               in shared memory and TMA stores, while the MMA warp already fills
 //               the other accumulator.
-// TMEM columns: accumulators [0, 192) and [192, 384); three scale buffers of 40
-// columns from 384: per K=64 step, 4 columns of A scales (row r at lane r%32,
-// column r/32) then 6 columns of W scales for the tile's 192 rows.
+// TMEM columns (each CTA): accumulators [0, 192) and [192, 384); three scale
+// buffers of 40 columns from 384: per K=64 step, 4 columns of A scales (row r
+// at lane r%32, column r/32) then 6 columns of W scales for the tile's 192 rows.
+// No TMA load uses cluster multicast; only tcgen05.commit is multicast.
 // Every mbarrier wait is bounded; on expiry the kernel sets the device error
 // word, stops issuing work, drains what it issued and frees its TMEM.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "fh_internal.h"
 
@@ -45,15 +54,12 @@ namespace {
 
 __device__ unsigned int g_device_error = 0;
 
-constexpr int BM = 128;
-constexpr int BN = 192;
+constexpr int BN = 192;                  // output columns per tile
 constexpr int BK = 256;                  // FP4 elements per stage = 128 bytes per row
 constexpr int kMmaK = 64;                // K of one tcgen05.mma kind::mxf4nvf4
 constexpr int kKSteps = BK / kMmaK;      // 4
-constexpr int kStages = 4;
-constexpr int kABytes = BM * BK / 2;     // 16384
-constexpr int kBBytes = BN * BK / 2;     // 24576
 constexpr int kAtomBytes = 512;          // 128 rows x 4 scales
+constexpr int kABytes = 128 * BK / 2;    // 16384: one CTA's 128 A rows
 constexpr int kSFABytes = kKSteps * kAtomBytes;      // 2048
 constexpr int kSFBBytes = 2 * kKSteps * kAtomBytes;  // 4096
 constexpr int kEpiWarps = 4;
@@ -67,28 +73,35 @@ constexpr int kAccCols = BN;
 constexpr int kSfCols = 4 * kKSteps + 6 * kKSteps;    // 40 per stage: A 4, W 6 per K=64 step
 constexpr int kSfBufs = 3;
 constexpr int kSfCol0 = 2 * kAccCols;                 // 384
-
-constexpr int kOffA = 0;
-constexpr int kOffB = kOffA + kStages * kABytes;
-constexpr int kOffSFA = kOffB + kStages * kBBytes;
-constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
-constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
-constexpr int kOffBias = kOffEpi + kEpiWarps * 2 * kEpiBufBytes;
-constexpr int kOffBar = kOffBias + kEpiWarps * BN * 4;
-// full, empty (per stage); acc full, acc empty (x2); scale full, scale empty (x3); drain
-constexpr int kNumBars = 2 * kStages + 4 + 2 * kSfBufs + 1;
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
-constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
-
-static_assert(kOffB % 1024 == 0 && kOffSFA % 1024 == 0 && kOffEpi % 1024 == 0, "alignment");
-static_assert(kSmemAlloc <= 232448, "shared memory budget");
 static_assert(kSfCol0 + kSfBufs * kSfCols <= kTmemCols, "TMEM budget");
 
-// Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format
-// 1), both K-major, UE4M3 scales, N >> 3 at bit 17, M >> 4 at bit 24, dense,
-// K = 64, scale-factor ids 0.
-constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+template <int kCta>
+struct Cfg {
+  static constexpr int BM = 128 * kCta;                // output rows per tile
+  static constexpr int kBRows = BN / kCta;             // W rows each CTA loads
+  static constexpr int kStages = kCta == 2 ? 5 : 4;
+  static constexpr int kBBytes = kBRows * BK / 2;
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kABytes;
+  static constexpr int kOffSFA = kOffB + kStages * kBBytes;
+  static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
+  static constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
+  static constexpr int kOffBias = kOffEpi + kEpiWarps * 2 * kEpiBufBytes;
+  static constexpr int kOffBar = kOffBias + kEpiWarps * BN * 4;
+  // full, empty, scale-smem (per stage); acc full, acc empty (x2); scale full,
+  // scale empty (x3); drain
+  static constexpr int kNumBars = 3 * kStages + 4 + 2 * kSfBufs + 1;
+  static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+  // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1
+  // (format 1), both K-major, UE4M3 scales, N >> 3 at bit 17, M >> 4 at bit
+  // 24, dense, K = 64, scale-factor ids 0.
+  static constexpr uint32_t kIdesc =
+      (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+  static_assert(kOffB % 1024 == 0 && kOffSFA % 1024 == 0 && kOffEpi % 1024 == 0, "alignment");
+  static_assert(kBBytes % 1024 == 0, "W stage alignment");
+  static_assert(kSmemAlloc <= 232448, "shared memory budget");
+};
 
 struct Params {
   const uint8_t* sfa;
@@ -99,10 +112,10 @@ struct Params {
   int n_tiles, num_tiles, k_stages;
   int ksteps_total;  // K / 64
   int sf_katoms;     // K / 64: 512-byte atoms per 128-row scale block
-  int n_sf_blocks;   // ceil(N / 128)
+  int n_sfa_blocks;  // ceil(M / 128)
+  int n_sfb_blocks;  // ceil(N / 128)
 };
 
-// ---- PTX wrappers ------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return (uint32_t)__cvta_generic_to_shared(p);
@@ -117,15 +130,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
@@ -158,13 +168,74 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
   return false;
 }
 
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
+// Tensor TMA load into this CTA's shared memory.  kCta == 2: `bar` may be the
+// leader CTA's barrier (a shared::cluster address); no multicast.
+template <int kCta>
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  if (kCta == 1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+  } else {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+        : "memory");
+  }
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+// Arrive (release at cluster scope) on a barrier given by its shared::cluster address.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// The leader CTA's copy of a barrier of this CTA: its shared::cluster address
+// for a pair, the barrier itself for a single CTA.
+template <int kCta>
+__device__ __forceinline__ uint32_t leader_bar(uint32_t local) {
+  return kCta == 2 ? map_to_rank(local, 0) : local;
+}
+
+template <int kCta>
+__device__ __forceinline__ void arrive_leader(uint32_t bar) {
+  if (kCta == 2)
+    mbar_arrive_cluster(bar);
+  else
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+template <int kCta>
+__device__ __forceinline__ void arrive_expect_tx_leader(uint32_t bar, uint32_t bytes) {
+  if (kCta == 2)
+    mbar_arrive_expect_tx_cluster(bar, bytes);
+  else
+    mbar_arrive_expect_tx(bar, bytes);
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
@@ -200,8 +271,24 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Arrive on `bar` (in this CTA, or at the same offset in every CTA of the
+// pair) once every tcgen05 operation this thread issued has completed.
+template <int kCta>
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+  if (kCta == 1) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+  } else {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            bar),
+        "h"((uint16_t)3)
+        : "memory");
+  }
+}
+
+__device__ __forceinline__ void tc_commit_local2(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
 }
 
@@ -217,15 +304,26 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, bool swizzle128) {
   return d;
 }
 
+template <int kCta>
 __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate,
                                        uint32_t sfa_tmem, uint32_t sfb_tmem) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
-      " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
+  if (kCta == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(Cfg<1>::kIdesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
+        " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(Cfg<2>::kIdesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+  }
 }
 
 // 32 consecutive TMEM columns of this thread's lane.
@@ -292,38 +390,47 @@ struct Ring {
   }
 };
 
+template <int kCta>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmY, const Params p) {
+  using C = Cfg<kCta>;
+  constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
-  const uint32_t bar0 = sbase + kOffBar;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };
-  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
-  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * kStages + a); };
-  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * kStages + 2 + a); };
-  auto sff_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 4 + b); };
-  auto sfe_bar = [&](int b) { return bar0 + 8u * (2 * kStages + 4 + kSfBufs + b); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * kStages + 4 + 2 * kSfBufs);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 8);
+  const uint32_t bar0 = sbase + C::kOffBar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };            // leader: A and W landed (both CTAs)
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };     // each CTA: stage free again
+  auto sfs_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };   // each CTA: its scale atoms landed
+  auto accf_bar = [&](int a) { return bar0 + 8u * (3 * S + a); };  // each CTA: accumulator ready
+  auto acce_bar = [&](int a) { return bar0 + 8u * (3 * S + 2 + a); };        // leader: accumulator drained
+  auto sff_bar = [&](int b) { return bar0 + 8u * (3 * S + 4 + b); };         // leader: scales staged
+  auto sfe_bar = [&](int b) { return bar0 + 8u * (3 * S + 4 + kSfBufs + b); };  // each CTA: scale buffer free
+  const uint32_t drain_bar = bar0 + 8u * (3 * S + 4 + 2 * kSfBufs);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + C::kNumBars * 8 + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kCta == 2 ? cluster_rank() : 0u;
+  const bool leader = rank == 0;
+  const int pair = kCta == 2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int npairs = kCta == 2 ? (int)(gridDim.x >> 1) : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full_bar(s), kCta);
       mbar_init(empty_bar(s), 1);
+      mbar_init(sfs_bar(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), kEpiWarps);
+      mbar_init(acce_bar(a), kEpiWarps * kCta);
     }
     for (int b = 0; b < kSfBufs; ++b) {
-      mbar_init(sff_bar(b), kSfWarps);
+      mbar_init(sff_bar(b), kSfWarps * kCta);
       mbar_init(sfe_bar(b), 1);
     }
     mbar_init(drain_bar, 1);
@@ -334,25 +441,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmY)) : "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    if (kCta == 1) {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                   "r"(kTmemCols));
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if (kCta == 2) cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ===================== TMA producer =====================
+    // ===================== TMA producer (every CTA) =====================
     if (lane == 0) {
       Ring st;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int t = pair; t < p.num_tiles && ok; t += npairs) {
         const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
-        const int m0 = m_tile * BM, n0 = n_tile * BN;
+        const int arow = m_tile * C::BM + (int)rank * 128;   // this CTA's A rows
+        const int n0 = n_tile * BN;
+        const int brow = n0 + (int)rank * C::kBRows;          // this CTA's W rows
+        const int ablk = arow / 128;
+        const bool has_sfa = ablk < p.n_sfa_blocks;
         const int jb0 = n0 / 128;
+        const int nsfb = (jb0 + 1 < p.n_sfb_blocks) ? 2 : 1;
         for (int kt = 0; kt < p.k_stages; ++kt) {
           if (!wait_bounded(empty_bar(st.slot), st.phase ^ 1u, abort_flag)) {
             ok = false;
@@ -360,36 +478,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
           const uint32_t sf_bytes = (uint32_t)ks * kAtomBytes;
-          const int nsfb = (jb0 + 1 < p.n_sf_blocks) ? 2 : 1;
-          const uint32_t fb = full_bar(st.slot);
-          mbar_arrive_expect_tx(fb, kABytes + kBBytes + sf_bytes * (1 + nsfb));
-          tma_load_2d(sbase + kOffA + st.slot * kABytes, &tmA, fb, kt * (BK / 2), m0);
-          tma_load_2d(sbase + kOffB + st.slot * kBBytes, &tmB, fb, kt * (BK / 2), n0);
+          const uint32_t fb = leader_bar<kCta>(full_bar(st.slot));
+          arrive_expect_tx_leader<kCta>(fb, kABytes + C::kBBytes);
+          tma_load_2d<kCta>(sbase + C::kOffA + st.slot * kABytes, &tmA, fb, kt * (BK / 2), arow);
+          tma_load_2d<kCta>(sbase + C::kOffB + st.slot * C::kBBytes, &tmB, fb, kt * (BK / 2), brow);
+          const uint32_t sb = sfs_bar(st.slot);
+          mbar_arrive_expect_tx(sb, sf_bytes * ((has_sfa ? 1u : 0u) + (uint32_t)nsfb));
           const size_t katom0 = (size_t)kt * kKSteps;
-          bulk_load(sbase + kOffSFA + st.slot * kSFABytes,
-                    p.sfa + ((size_t)m_tile * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, fb);
+          if (has_sfa)
+            bulk_load(sbase + C::kOffSFA + st.slot * kSFABytes,
+                      p.sfa + ((size_t)ablk * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
           for (int r = 0; r < nsfb; ++r)
-            bulk_load(sbase + kOffSFB + st.slot * kSFBBytes + r * (kKSteps * kAtomBytes),
-                      p.sfb + ((size_t)(jb0 + r) * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, fb);
-          st.next(kStages);
+            bulk_load(sbase + C::kOffSFB + st.slot * kSFBBytes + r * (kKSteps * kAtomBytes),
+                      p.sfb + ((size_t)(jb0 + r) * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
+          st.next(S);
         }
       }
-      // Drain: wait until every load this thread issued has landed, so no
-      // copy still targets shared memory when the CTA retires.
-      for (int s = 0; s < kStages; ++s) {
-        // Stage s was last filled in the phase before `phase` if s >= slot.
+      // Drain: wait until every load this thread issued into its own shared
+      // memory has landed (the scale atoms here; the leader also sees A and W
+      // of both CTAs land on its stage barriers).
+      for (int s = 0; s < S; ++s) {
         const uint32_t par = (s < st.slot) ? st.phase : (st.phase ^ 1u);
-        wait_bounded(full_bar(s), par, abort_flag);
+        wait_bounded(sfs_bar(s), par, abort_flag);
+        if (leader) wait_bounded(full_bar(s), par, abort_flag);
       }
     }
   } else if (warp == 1) {
-    // ===================== MMA issuer =====================
-    if (lane == 0) {
+    // ===================== MMA issuer (leader CTA) =====================
+    if (lane == 0 && leader) {
       Ring st, sf;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int t = pair; t < p.num_tiles && ok; t += npairs) {
         if (!wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
@@ -401,48 +522,51 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
-          const uint32_t a_addr = sbase + kOffA + st.slot * kABytes;
-          const uint32_t b_addr = sbase + kOffB + st.slot * kBBytes;
+          const uint32_t a_addr = sbase + C::kOffA + st.slot * kABytes;
+          const uint32_t b_addr = sbase + C::kOffB + st.slot * C::kBBytes;
           const uint32_t sf_tmem = tmem_base + (uint32_t)(kSfCol0 + sf.slot * kSfCols);
           for (int k = 0; k < ks; ++k) {
-            tc_mma(d_tmem, smem_desc(a_addr + k * (kMmaK / 2), true), smem_desc(b_addr + k * (kMmaK / 2), true),
-                   (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
+            tc_mma<kCta>(d_tmem, smem_desc(a_addr + k * (kMmaK / 2), true), smem_desc(b_addr + k * (kMmaK / 2), true),
+                         (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
           }
-          tc_commit(empty_bar(st.slot));  // the stage's shared memory, once these MMAs have read it
-          tc_commit(sfe_bar(sf.slot));    // the scale buffer, likewise
-          st.next(kStages);
+          tc_commit<kCta>(empty_bar(st.slot));  // the stage's shared memory (both CTAs), once read
+          tc_commit<kCta>(sfe_bar(sf.slot));    // the scale buffers (both CTAs), likewise
+          st.next(S);
           sf.next(kSfBufs);
         }
         if (!ok) break;
-        tc_commit(accf_bar(acc));  // accumulator ready for the epilogue
+        tc_commit<kCta>(accf_bar(acc));  // accumulator ready for both CTAs' epilogues
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // Drain: every MMA issued above has completed before TMEM is released.
-      tc_commit(drain_bar);
+      if (kCta == 1)
+        tc_commit<1>(drain_bar);
+      else
+        tc_commit_local2(drain_bar);
       wait_bounded(drain_bar, 0, abort_flag);
     }
   } else if (warp >= kFirstSfWarp) {
-    // ===================== scale stagers =====================
+    // ===================== scale stagers (every CTA) =====================
     // Lane l of the warp for quadrant q writes TMEM lane 32q + l.  A scale atom
     // holds, at bytes 16 l .. 16 l + 15, the four K=64 scales of rows l, l+32,
     // l+64, l+96: TMEM columns 0..3 of a K step (row r at column r/32).
     const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
     Ring st, sf;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+    for (int t = pair; t < p.num_tiles && ok; t += npairs) {
       const bool odd = ((t % p.n_tiles) * BN) % 128 != 0;  // tile starts at row 64 of a scale block
       for (int kt = 0; kt < p.k_stages; ++kt) {
-        if (!wait_bounded(full_bar(st.slot), st.phase, abort_flag) ||
+        if (!wait_bounded(sfs_bar(st.slot), st.phase, abort_flag) ||
             !wait_bounded(sfe_bar(sf.slot), sf.phase ^ 1u, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sfa_addr = sbase + kOffSFA + st.slot * kSFABytes + lane * 16;
-        const uint32_t sfb_addr = sbase + kOffSFB + st.slot * kSFBBytes + lane * 16;
+        const uint32_t sfa_addr = sbase + C::kOffSFA + st.slot * kSFABytes + lane * 16;
+        const uint32_t sfb_addr = sbase + C::kOffSFB + st.slot * kSFBBytes + lane * 16;
         uint32_t va[16], vb[24];
 #pragma unroll
         for (int k = 0; k < kKSteps; ++k) {
@@ -476,23 +600,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(sff_bar(sf.slot));
-        st.next(kStages);
+        if (lane == 0) arrive_leader<kCta>(leader_bar<kCta>(sff_bar(sf.slot)));
+        st.next(S);
         sf.next(kSfBufs);
       }
     }
   } else {
-    // ===================== epilogue =====================
+    // ===================== epilogue (every CTA) =====================
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    uint8_t* stage_buf = smem + kOffEpi + (warp - 2) * 2 * kEpiBufBytes;
-    float* bias_s = reinterpret_cast<float*>(smem + kOffBias) + (warp - 2) * BN;
+    uint8_t* stage_buf = smem + C::kOffEpi + (warp - 2) * 2 * kEpiBufBytes;
+    float* bias_s = reinterpret_cast<float*>(smem + C::kOffBias) + (warp - 2) * BN;
     int acc = 0;
     uint32_t acc_phase = 0;
     int buf = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+    for (int t = pair; t < p.num_tiles; t += npairs) {
       const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
-      const int m0 = m_tile * BM, n0 = n_tile * BN;
+      const int row0 = m_tile * C::BM + (int)rank * 128 + 32 * q;  // this warp's 32 output rows
+      const int n0 = n_tile * BN;
       // The tile's bias, in FP32, staged in this warp's shared memory before
       // the accumulator is ready (lanes 0..23 load 8 values each).
       if (lane < BN / 8) {
@@ -543,16 +668,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0 && m0 + 32 * q < p.M) {  // rows past M: nothing to store
-          tma_store_2d(&tmY, smem_u32(sb), col0, m0 + 32 * q);
-        }
+        if (lane == 0 && row0 < p.M) tma_store_2d(&tmY, smem_u32(sb), col0, row0);  // rows past M: nothing to store
         if (lane == 0) bulk_commit();
         buf ^= 1;
       }
       // All TMEM reads of this accumulator are done: hand it back to the MMA warp.
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (lane == 0) arrive_leader<kCta>(leader_bar<kCta>(acce_bar(acc)));
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;
@@ -564,10 +687,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (kCta == 2) cluster_sync();  // the peer no longer needs this CTA's shared memory or TMEM
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+    if (kCta == 1)
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+    else
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
   }
 }
 
@@ -603,6 +730,67 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Which kernel form to run: the CTA pair (default) or single CTAs.  The
+// environment variable FH_GEMM_CTAS=1 selects the single-CTA form (both run the
+// same arithmetic; the switch exists to compare them).
+int cta_mode() {
+  static int mode = 0;
+  if (mode == 0) {
+    const char* e = getenv("FH_GEMM_CTAS");
+    mode = (e != nullptr && e[0] == '1') ? 1 : 2;
+  }
+  return mode;
+}
+
+template <int kCta>
+cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const Params& p,
+                        cudaStream_t s) {
+  using C = Cfg<kCta>;
+  static int configured_device = -1;
+  static int max_groups = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e =
+        cudaFuncSetAttribute(nvfp4_linear_kernel<kCta>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+    if (e != cudaSuccess) return e;
+    max_groups = sm_count() / kCta;
+    if (kCta == 2) {
+      // Clusters that fit at once (an SM left without a partner cannot host one).
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * max_groups);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = C::kSmemAlloc;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4_linear_kernel<2>, &cfg) == cudaSuccess && clusters > 0)
+        max_groups = clusters < max_groups ? clusters : max_groups;
+      cudaGetLastError();
+    }
+    configured_device = dev;
+  }
+  const int groups = p.num_tiles < max_groups ? p.num_tiles : max_groups;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCta;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(groups * kCta);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmemAlloc;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = kCta == 2 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta>, tmA, tmB, tmY, p);
+}
+
 }  // namespace
 
 cudaError_t read_and_clear_device_error(unsigned int* bits, cudaStream_t s) {
@@ -620,13 +808,14 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
                                 const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
                                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
                                 cudaStream_t s, const char** why) {
+  const int ctas = cta_mode();
   CUtensorMap tmA, tmB, tmY;
-  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M,
-                   (uint64_t)K / 2, BK / 2, BM) ||
-      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N,
-                   (uint64_t)K / 2, BK / 2, BN) ||
-      !make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
-                   (uint64_t)N * 2, kEpiCols, 32)) {
+  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
+                   BK / 2, 128) ||
+      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                   BK / 2, BN / ctas) ||
+      !make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
+                   kEpiCols, 32)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or a layout rule violated)";
     return cudaErrorNotSupported;
   }
@@ -638,26 +827,16 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
   p.M = (int)M;
   p.N = (int)N;
   p.K = (int)K;
-  const int m_tiles = (int)((M + BM - 1) / BM);
+  const int bm = 128 * ctas;
+  const int m_tiles = (int)((M + bm - 1) / bm);
   p.n_tiles = (int)((N + BN - 1) / BN);
   p.num_tiles = m_tiles * p.n_tiles;
   p.k_stages = (int)((K + BK - 1) / BK);
   p.ksteps_total = (int)(K / kMmaK);
   p.sf_katoms = (int)(K / kMmaK);
-  p.n_sf_blocks = (int)((N + 127) / 128);
-
-  static int configured_device = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(nvfp4_linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
-  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
-  nvfp4_linear_kernel<<<grid, kThreads, kSmemAlloc, s>>>(tmA, tmB, tmY, p);
-  return cudaGetLastError();
+  p.n_sfa_blocks = (int)((M + 127) / 128);
+  p.n_sfb_blocks = (int)((N + 127) / 128);
+  return ctas == 2 ? launch_form<2>(tmA, tmB, tmY, p, s) : launch_form<1>(tmA, tmB, tmY, p, s);
 }
 
 }  // namespace fh

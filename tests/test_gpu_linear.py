@@ -138,3 +138,16 @@ def test_back_to_back_calls_reuse_nothing():
     assert torch.equal(ya.view(torch.int16), ya2.view(torch.int16))
     check_linear(yb, x2, 0.01, w2, 0.0001, None)
     fh().fh_device_status()
+
+
+def test_single_cta_form_matches_oracle():
+    """The single-CTA kernel form (FH_GEMM_CTAS=1: 128-row tiles, cta_group::1)
+    passes the same parity cases as the default CTA-pair form."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, FH_GEMM_CTAS="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", os.path.abspath(__file__),
+                        "-k", "small or tiny or no_bias or back_to_back or full_size"],
+                       env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
