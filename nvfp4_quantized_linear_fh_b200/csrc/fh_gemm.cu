@@ -79,14 +79,15 @@ template <int kCta>
 struct Cfg {
   static constexpr int BM = 128 * kCta;                // output rows per tile
   static constexpr int kBRows = BN / kCta;             // W rows each CTA loads
-  static constexpr int kStages = kCta == 2 ? 5 : 4;
+  static constexpr int kStages = kCta == 2 ? 6 : 4;
+  static constexpr int kEpiBufs = kCta == 2 ? 1 : 2;   // output staging buffers per epilogue warp
   static constexpr int kBBytes = kBRows * BK / 2;
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kABytes;
   static constexpr int kOffSFA = kOffB + kStages * kBBytes;
   static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
   static constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
-  static constexpr int kOffBias = kOffEpi + kEpiWarps * 2 * kEpiBufBytes;
+  static constexpr int kOffBias = kOffEpi + kEpiWarps * kEpiBufs * kEpiBufBytes;
   static constexpr int kOffBar = kOffBias + kEpiWarps * BN * 4;
   // full, empty, scale-smem (per stage); acc full, acc empty (x2); scale full,
   // scale empty (x3); drain
@@ -135,12 +136,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+// One lane of the (converged) warp; the whole warp runs the issuing loops so
+// that every operand of the tcgen05 / TMA instructions stays warp-uniform.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
 }
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -194,14 +207,14 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t local, uint32_t rank) {
   return r;
 }
 
-// Arrive (release at cluster scope) on a barrier given by its shared::cluster address.
+// Arrive on a barrier given by its shared::cluster address (possibly in the
+// peer CTA).
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t cluster_bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.release.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar),
-               "r"(bytes)
+  asm volatile("mbarrier.arrive.expect_tx.shared::cluster.b64 _, [%0], %1;" ::"r"(cluster_bar), "r"(bytes)
                : "memory");
 }
 
@@ -255,6 +268,9 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 __device__ __forceinline__ void bulk_wait_read_1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
@@ -459,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ===================== TMA producer (every CTA) =====================
-    if (lane == 0) {
+    {
       Ring st;
       bool ok = true;
       for (int t = pair; t < p.num_tiles && ok; t += npairs) {
@@ -472,25 +488,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int jb0 = n0 / 128;
         const int nsfb = (jb0 + 1 < p.n_sfb_blocks) ? 2 : 1;
         for (int kt = 0; kt < p.k_stages; ++kt) {
-          if (!wait_bounded(empty_bar(st.slot), st.phase ^ 1u, abort_flag)) {
+          if (!__all_sync(0xFFFFFFFFu, wait_bounded(empty_bar(st.slot), st.phase ^ 1u, abort_flag))) {
             ok = false;
             break;
           }
           const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
           const uint32_t sf_bytes = (uint32_t)ks * kAtomBytes;
           const uint32_t fb = leader_bar<kCta>(full_bar(st.slot));
-          arrive_expect_tx_leader<kCta>(fb, kABytes + C::kBBytes);
-          tma_load_2d<kCta>(sbase + C::kOffA + st.slot * kABytes, &tmA, fb, kt * (BK / 2), arow);
-          tma_load_2d<kCta>(sbase + C::kOffB + st.slot * C::kBBytes, &tmB, fb, kt * (BK / 2), brow);
           const uint32_t sb = sfs_bar(st.slot);
-          mbar_arrive_expect_tx(sb, sf_bytes * ((has_sfa ? 1u : 0u) + (uint32_t)nsfb));
           const size_t katom0 = (size_t)kt * kKSteps;
-          if (has_sfa)
-            bulk_load(sbase + C::kOffSFA + st.slot * kSFABytes,
-                      p.sfa + ((size_t)ablk * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
-          for (int r = 0; r < nsfb; ++r)
-            bulk_load(sbase + C::kOffSFB + st.slot * kSFBBytes + r * (kKSteps * kAtomBytes),
-                      p.sfb + ((size_t)(jb0 + r) * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
+          if (elect_one()) {
+            arrive_expect_tx_leader<kCta>(fb, kABytes + C::kBBytes);
+            tma_load_2d<kCta>(sbase + C::kOffA + st.slot * kABytes, &tmA, fb, kt * (BK / 2), arow);
+            tma_load_2d<kCta>(sbase + C::kOffB + st.slot * C::kBBytes, &tmB, fb, kt * (BK / 2), brow);
+            mbar_arrive_expect_tx(sb, sf_bytes * ((has_sfa ? 1u : 0u) + (uint32_t)nsfb));
+            if (has_sfa)
+              bulk_load(sbase + C::kOffSFA + st.slot * kSFABytes,
+                        p.sfa + ((size_t)ablk * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
+            for (int r = 0; r < nsfb; ++r)
+              bulk_load(sbase + C::kOffSFB + st.slot * kSFBBytes + r * (kKSteps * kAtomBytes),
+                        p.sfb + ((size_t)(jb0 + r) * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
+          }
+          __syncwarp();
           st.next(S);
         }
       }
@@ -505,47 +524,65 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ===================== MMA issuer (leader CTA) =====================
-    if (lane == 0 && leader) {
+    if (leader) {
       Ring st, sf;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      // Descriptors of stage 0, K step 0; a stage or K step moves the start
+      // address field (16-byte units) by a constant.
+      const uint64_t adesc0 = smem_desc(sbase + C::kOffA, true);
+      const uint64_t bdesc0 = smem_desc(sbase + C::kOffB, true);
       for (int t = pair; t < p.num_tiles && ok; t += npairs) {
-        if (!wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag)) break;
+        if (!__all_sync(0xFFFFFFFFu, wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
         for (int kt = 0; kt < p.k_stages; ++kt) {
-          if (!wait_bounded(full_bar(st.slot), st.phase, abort_flag) ||
-              !wait_bounded(sff_bar(sf.slot), sf.phase, abort_flag)) {
+          const bool landed = wait_bounded(full_bar(st.slot), st.phase, abort_flag) &&
+                              wait_bounded(sff_bar(sf.slot), sf.phase, abort_flag);
+          if (!__all_sync(0xFFFFFFFFu, landed)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
-          const uint32_t a_addr = sbase + C::kOffA + st.slot * kABytes;
-          const uint32_t b_addr = sbase + C::kOffB + st.slot * C::kBBytes;
+          const uint64_t adesc = adesc0 + (uint64_t)((st.slot * kABytes) >> 4);
+          const uint64_t bdesc = bdesc0 + (uint64_t)((st.slot * C::kBBytes) >> 4);
           const uint32_t sf_tmem = tmem_base + (uint32_t)(kSfCol0 + sf.slot * kSfCols);
-          for (int k = 0; k < ks; ++k) {
-            tc_mma<kCta>(d_tmem, smem_desc(a_addr + k * (kMmaK / 2), true), smem_desc(b_addr + k * (kMmaK / 2), true),
-                         (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
+          if (elect_one()) {
+            if (ks == kKSteps) {
+#pragma unroll
+              for (int k = 0; k < kKSteps; ++k)
+                tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
+                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
+            } else {
+              for (int k = 0; k < ks; ++k)
+                tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
+                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
+            }
+            tc_commit<kCta>(empty_bar(st.slot));  // the stage's shared memory (both CTAs), once read
+            tc_commit<kCta>(sfe_bar(sf.slot));    // the scale buffers (both CTAs), likewise
           }
-          tc_commit<kCta>(empty_bar(st.slot));  // the stage's shared memory (both CTAs), once read
-          tc_commit<kCta>(sfe_bar(sf.slot));    // the scale buffers (both CTAs), likewise
+          __syncwarp();
           st.next(S);
           sf.next(kSfBufs);
         }
         if (!ok) break;
-        tc_commit<kCta>(accf_bar(acc));  // accumulator ready for both CTAs' epilogues
+        if (elect_one()) tc_commit<kCta>(accf_bar(acc));  // accumulator ready for both CTAs' epilogues
+        __syncwarp();
         if (++acc == 2) {
           acc = 0;
           acc_phase ^= 1u;
         }
       }
       // Drain: every MMA issued above has completed before TMEM is released.
-      if (kCta == 1)
-        tc_commit<1>(drain_bar);
-      else
-        tc_commit_local2(drain_bar);
+      if (elect_one()) {
+        if (kCta == 1)
+          tc_commit<1>(drain_bar);
+        else
+          tc_commit_local2(drain_bar);
+      }
+      __syncwarp();
       wait_bounded(drain_bar, 0, abort_flag);
     }
   } else if (warp >= kFirstSfWarp) {
@@ -609,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================== epilogue (every CTA) =====================
     const int q = warp & 3;  // TMEM lane quadrant this warp may access
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    uint8_t* stage_buf = smem + C::kOffEpi + (warp - 2) * 2 * kEpiBufBytes;
+    uint8_t* stage_buf = smem + C::kOffEpi + (warp - 2) * C::kEpiBufs * kEpiBufBytes;
     float* bias_s = reinterpret_cast<float*>(smem + C::kOffBias) + (warp - 2) * BN;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -656,7 +693,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           packed[2 * j + 1] = pack_bf16x2(y2, y3);
         }
         // Reuse a staging buffer only after its previous TMA store has read it.
-        if (lane == 0) bulk_wait_read_1();
+        if (lane == 0) {
+          if (C::kEpiBufs == 1)
+            bulk_wait_read_0();
+          else
+            bulk_wait_read_1();
+        }
         __syncwarp();
         uint8_t* sb = stage_buf + buf * kEpiBufBytes;
         const uint32_t row = (uint32_t)lane;
@@ -670,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0 && row0 < p.M) tma_store_2d(&tmY, smem_u32(sb), col0, row0);  // rows past M: nothing to store
         if (lane == 0) bulk_commit();
-        buf ^= 1;
+        if (C::kEpiBufs == 2) buf ^= 1;
       }
       // All TMEM reads of this accumulator are done: hand it back to the MMA warp.
       tc_fence_before();
