@@ -183,9 +183,11 @@ int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t 
 int fh_device_status(fh_stream_t stream) {
   g_last_error[0] = 0;
   if (int st = check_device()) return st;
-  unsigned int bits = 0;
+  unsigned int bits = 0, qbits = 0;
   cudaError_t e = fh::read_and_clear_device_error(&bits, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = fh::read_and_clear_quant_error(&qbits);
   if (e != cudaSuccess) return cuda_fail(e, "fh_device_status");
+  bits |= qbits;
   if (bits & fh::kDevErrTimeout)
     return fail(FH_ERR_TIMEOUT, "a kernel gave up on a bounded on-chip wait%s");
   return FH_OK;

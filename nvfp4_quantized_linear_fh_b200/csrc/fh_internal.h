@@ -16,6 +16,8 @@ enum : unsigned int {
 // Host side: synchronize `s`, then read and clear the device error word of the
 // current device (fh_gemm.cu owns the word).
 cudaError_t read_and_clear_device_error(unsigned int* bits, cudaStream_t s);
+// The quantizer's error word (fh_quant.cu); call after the stream is synchronized.
+cudaError_t read_and_clear_quant_error(unsigned int* bits);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();

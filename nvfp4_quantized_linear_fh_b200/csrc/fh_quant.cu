@@ -42,7 +42,6 @@ namespace fh {
 
 namespace {
 
-constexpr int kQuantThreads = 256;
 constexpr uint32_t kBf16Inf = 0x7F80u;
 
 struct __align__(16) QuantTable {
@@ -62,7 +61,12 @@ struct QuantParams {
   int64_t M, K, ldx;
   float inv6sg;       // 1 / (6 s_g): scale-code candidate multiplier
   uint32_t clip_thr;  // smallest BF16 magnitude strictly beyond 2688 s_g
-  int wide;           // 32-byte loads allowed
+  // Streaming units: R rows x kc columns (kc divides K), at most 8192 elements.
+  int64_t kc, R, col_units, n_units;
+  int nbu;            // 16-element blocks per unit row: kc / 16
+  int step_rows;      // consumer stride in blocks (256) as whole rows ...
+  int step_blocks;    // ... plus remaining blocks: 256 = step_rows * nbu + step_blocks
+  int one_copy;       // rows of a unit are contiguous in x: one bulk copy per unit
 };
 
 // ---- host: the exact decision table for one global scale ----------------------
@@ -239,22 +243,6 @@ __device__ __forceinline__ void codes_fast(float inv, const uint32_t* w, uint32_
   out[1] = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
 }
 
-__device__ __forceinline__ void load_block(const uint16_t* p, uint32_t* w, bool wide) {
-  if (wide) {
-    asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]),
-                   "=r"(w[6]), "=r"(w[7])
-                 : "l"(p));
-  } else {
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
-                 : "l"(p));
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(w[4]), "=r"(w[5]), "=r"(w[6]), "=r"(w[7])
-                 : "l"(p + 8));
-  }
-}
-
 __device__ __forceinline__ int64_t tiled_offset(int64_t m, int64_t s, int64_t katoms) {
   return ((m >> 7) * katoms + (s >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (s & 3);
 }
@@ -308,52 +296,163 @@ __device__ __forceinline__ void store_scale(const QuantParams& p, uint32_t sc, b
   }
 }
 
+// Streaming layout of the quantizer: one producer warp moves units of at most
+// 8192 BF16 elements (R rows x kc columns, 16 KB) from HBM into a ring of
+// shared-memory stages with bulk asynchronous copies; eight consumer warps
+// quantize each unit from shared memory, one 16-element block per thread per
+// pass.  Two CTAs per SM keep ~190 KB of loads in flight per SM.
+constexpr int kQConsumerWarps = 8;
+constexpr int kQThreads = 32 * (kQConsumerWarps + 1);
+constexpr int kQStages = 6;
+constexpr int kQUnitElems = 8192;
+constexpr int kQUnitBytes = 2 * kQUnitElems;
+constexpr int kQSmem = kQStages * kQUnitBytes + 2 * 8 * kQStages + 64;
+
+__device__ unsigned int g_quant_error = 0;
+
+__device__ __forceinline__ uint32_t q_smem_u32(const void* ptr) { return (uint32_t)__cvta_generic_to_shared(ptr); }
+
+__device__ __forceinline__ bool q_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait (about 4 s, or until another warp of the CTA gave up).
+__device__ __forceinline__ bool q_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (q_try_wait(bar, parity)) return true;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t i = 1; i < (1u << 30); ++i) {
+    if (q_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u) {
+      if (*abort) return false;
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > 4000000000ull) break;
+    }
+  }
+  atomicOr(&g_quant_error, 1u);
+  *abort = 1;
+  return false;
+}
+
 // kGather4: K/16 % 4 == 0, so lanes 4i..4i+3 own four consecutive scales of
 // one row and store them as one word.
 template <bool kTiled, bool kGather4>
-__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_constant__ QuantParams p) {
+__global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_constant__ QuantParams p) {
+  extern __shared__ __align__(128) uint8_t qsmem[];
   __shared__ QuantTable tab;
   __shared__ unsigned long long cta_clips;
+  __shared__ int abort_flag_s;
+  volatile int* abort_flag = &abort_flag_s;
+  const uint32_t stage0 = q_smem_u32(qsmem);
+  const uint32_t bar0 = stage0 + kQStages * kQUnitBytes;
+  auto full_bar = [&](int st) { return bar0 + 8u * st; };
+  auto empty_bar = [&](int st) { return bar0 + 8u * (kQStages + st); };
   {
     const uint4* src = reinterpret_cast<const uint4*>(&p.tab);
     uint4* dst = reinterpret_cast<uint4*>(&tab);
     for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 16); i += blockDim.x) dst[i] = src[i];
   }
-  if (threadIdx.x == 0) cta_clips = 0;
+  if (threadIdx.x == 0) {
+    cta_clips = 0;
+    abort_flag_s = 0;
+    for (int st = 0; st < kQStages; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full_bar(st)));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty_bar(st)), "r"(kQConsumerWarps));
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
   __syncthreads();
 
-  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nb = p.K >> 4;
-  const int64_t total = p.M * nb;
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t katoms = nb >> 2;
-  const int64_t dm = (2 * stride) / nb, ds = (2 * stride) % nb;
-  int64_t base = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31);
-  // (m0, s0): this lane's first block of the step; (m1, s1): the second, one stride later.
-  int64_t m0 = (base + lane) / nb, s0 = (base + lane) % nb;
-  int64_t m1 = (base + stride + lane) / nb, s1 = (base + stride + lane) % nb;
   unsigned long long clips = 0;
 
-  for (; base < total; base += 2 * stride) {
-    const bool v0 = base + lane < total, v1 = base + stride + lane < total;
-    uint32_t w0[8], w1[8];
-    if (v0) load_block(p.x + m0 * p.ldx + 16 * s0, w0, p.wide);
-    if (v1) load_block(p.x + m1 * p.ldx + 16 * s1, w1, p.wide);
-    const uint32_t sc0 = v0 ? quantize_block(tab, p, w0, m0, s0, clips) : 0u;
-    const uint32_t sc1 = v1 ? quantize_block(tab, p, w1, m1, s1, clips) : 0u;
-    store_scale<kTiled, kGather4>(p, sc0, v0, lane, m0, s0, nb, katoms);
-    store_scale<kTiled, kGather4>(p, sc1, v1, lane, m1, s1, nb, katoms);
-    s0 += ds;
-    m0 += dm;
-    if (s0 >= nb) {
-      s0 -= nb;
-      ++m0;
+  if (warp == kQConsumerWarps) {
+    // ===== producer: bulk copies of whole units into the stage ring =====
+    if (lane == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        if (!q_wait(empty_bar(st), ph ^ 1u, abort_flag)) break;
+        const int64_t rb = u / p.col_units, cb = u % p.col_units;
+        const int64_t r0 = rb * p.R;
+        const int64_t rows = min(p.R, p.M - r0);
+        const uint32_t row_bytes = (uint32_t)(p.kc * 2);
+        const uint32_t dst = stage0 + st * kQUnitBytes;
+        const uint16_t* src = p.x + r0 * p.ldx + cb * p.kc;
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full_bar(st)),
+                     "r"((uint32_t)rows * row_bytes)
+                     : "memory");
+        if (p.one_copy) {
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+              "l"(src), "r"((uint32_t)rows * row_bytes), "r"(full_bar(st))
+              : "memory");
+        } else {
+          for (int64_t r = 0; r < rows; ++r)
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                    dst + (uint32_t)r * row_bytes),
+                "l"(src + r * p.ldx), "r"(row_bytes), "r"(full_bar(st))
+                : "memory");
+        }
+        if (++st == kQStages) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+      // Drain: every copy this thread issued has landed before the CTA retires.
+      for (int i = 0; i < kQStages; ++i) q_wait(full_bar(i), (i < st) ? ph : (ph ^ 1u), abort_flag);
     }
-    s1 += ds;
-    m1 += dm;
-    if (s1 >= nb) {
-      s1 -= nb;
-      ++m1;
+  } else {
+    // ===== consumers =====
+    const int ctid = threadIdx.x;  // 0 .. 255
+    const int64_t ublocks = p.R * p.nbu;  // blocks in a full unit
+    int st = 0;
+    uint32_t ph = 0;
+    for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      if (!q_wait(full_bar(st), ph, abort_flag)) break;
+      const int64_t rb = u / p.col_units, cb = u % p.col_units;
+      const int64_t r0 = rb * p.R;
+      const uint8_t* unit = qsmem + st * kQUnitBytes;
+      // This thread's blocks i = ctid, ctid + 256, ...: (row r, block sb) inside the unit.
+      int r = ctid / p.nbu, sb = ctid % p.nbu;
+      for (int64_t i0 = 0; i0 < ublocks; i0 += 32 * kQConsumerWarps) {
+        const int64_t i = i0 + ctid;
+        const int64_t m = r0 + r;
+        const int64_t sg = cb * p.nbu + sb;  // block index within the row
+        const bool valid = (i < ublocks) && (m < p.M);
+        uint32_t sc = 0;
+        if (valid) {
+          const uint4 q0 = *reinterpret_cast<const uint4*>(unit + 32 * i);
+          const uint4 q1 = *reinterpret_cast<const uint4*>(unit + 32 * i + 16);
+          const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          sc = quantize_block(tab, p, w, m, sg, clips);
+        }
+        store_scale<kTiled, kGather4>(p, sc, valid, lane, m, sg, nb, katoms);
+        r += p.step_rows;
+        sb += p.step_blocks;
+        if (sb >= p.nbu) {
+          sb -= p.nbu;
+          ++r;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
+      if (++st == kQStages) {
+        st = 0;
+        ph ^= 1u;
+      }
     }
   }
 
@@ -361,7 +460,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const __grid_co
     // Zero the scales of the padding rows M .. ceil(M/128)*128 - 1.
     const int64_t mpad = ((p.M + 127) >> 7) << 7;
     const int64_t npad = (mpad - p.M) * nb;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += stride)
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += (int64_t)gridDim.x * blockDim.x)
       p.scales[tiled_offset(p.M + i / nb, i % nb, katoms)] = 0;
   }
 
@@ -477,27 +576,59 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   p.K = K;
   p.ldx = ldx;
   p.inv6sg = (float)(1.0 / (6.0 * (double)sg));
-  p.wide = ((reinterpret_cast<uintptr_t>(x) & 31) == 0) && ((ldx % 16) == 0);
+  // Streaming units: kc = K if a row fits in a unit, else the largest divisor of
+  // K that is a multiple of 64 (16 without the four-scale gather) and fits.
+  {
+    const int64_t gran = (K % 64 == 0) ? 64 : 16;
+    int64_t kc = K;
+    if (K > kQUnitElems) {
+      kc = gran;
+      for (int64_t c = (kQUnitElems / gran) * gran; c >= gran; c -= gran)
+        if (K % c == 0) {
+          kc = c;
+          break;
+        }
+    }
+    p.kc = kc;
+    p.R = kQUnitElems / kc;
+    p.col_units = K / kc;
+    p.n_units = ((M + p.R - 1) / p.R) * p.col_units;
+    p.nbu = (int)(kc / 16);
+    p.step_rows = (32 * kQConsumerWarps) / p.nbu;
+    p.step_blocks = (32 * kQConsumerWarps) % p.nbu;
+    p.one_copy = (ldx == K && kc == K) ? 1 : 0;
+  }
   // Exact clip threshold: smallest BF16 magnitude strictly beyond 2688 * s_g
   // (2688 * s_g is exact in FP64: 5 + 24 significant bits).
   p.clip_thr = bf16_threshold(2688.0 * (double)sg, true);
-  const int64_t nb = K / 16;
   const bool tiled = layout == FH_SCALES_MMA_TILED;
-  const bool gather4 = (nb % 4) == 0;
-  const int64_t mpad = tiled ? ((M + 127) / 128) * 128 : M;
-  const int grid = grid_for((mpad * nb + 1) / 2, kQuantThreads, 4);
-  if (tiled) {
-    if (gather4)
-      quantize_kernel<true, true><<<grid, kQuantThreads, 0, s>>>(p);
-    else
-      quantize_kernel<true, false><<<grid, kQuantThreads, 0, s>>>(p);
-  } else {
-    if (gather4)
-      quantize_kernel<false, true><<<grid, kQuantThreads, 0, s>>>(p);
-    else
-      quantize_kernel<false, false><<<grid, kQuantThreads, 0, s>>>(p);
-  }
-  return cudaGetLastError();
+  const bool gather4 = (K / 16) % 4 == 0;
+  const int64_t want = p.n_units > 0 ? p.n_units : 1;
+  const int grid = (int)(want < 2 * (int64_t)sm_count() ? want : 2 * (int64_t)sm_count());
+  auto launch = [&](auto kernel, int& configured) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (configured != dev) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+      if (e != cudaSuccess) return e;
+      configured = dev;
+    }
+    kernel<<<grid, kQThreads, kQSmem, s>>>(p);
+    return cudaGetLastError();
+  };
+  static int cfg_tt = -1, cfg_tf = -1, cfg_ft = -1, cfg_ff = -1;
+  if (tiled)
+    return gather4 ? launch(quantize_kernel<true, true>, cfg_tt) : launch(quantize_kernel<true, false>, cfg_tf);
+  return gather4 ? launch(quantize_kernel<false, true>, cfg_ft) : launch(quantize_kernel<false, false>, cfg_ff);
+}
+
+cudaError_t read_and_clear_quant_error(unsigned int* bits) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_quant_error, sizeof v);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbol(g_quant_error, &zero, sizeof zero);
+  *bits = v;
+  return e;
 }
 
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, float* amax,
