@@ -140,27 +140,43 @@ void build_table(float sg_f, QuantTable* t) {
   }
   // Converter path check at both sides of every boundary and at the ends of the
   // BF16 range.  Negative inputs give the same magnitude with the sign bit set.
+  // When the FP32 product of a boundary value lands on a midpoint the nearest
+  // multiplier fails the check; a neighbouring FP32 multiplier usually passes,
+  // so up to two on each side are tried before the code falls back to the
+  // exact threshold path.
   for (int c = 0; c < 127; ++c) {
-    bool ok = true;
     auto exact_mag = [&](uint32_t a) {
       uint32_t m = 0;
       for (int j = 0; j < 7; ++j) m += (a >= t->code_thr[c][j]) ? 1u : 0u;
       return m;
     };
-    auto probe = [&](uint32_t a) {
-      const float y = bf16_bits_value(a) * t->inv[c];  // the kernel's FP32 multiply
-      ok = ok && converter_e2m1(y) == exact_mag(a);
+    auto passes = [&](float inv) {
+      bool ok = true;
+      auto probe = [&](uint32_t a) {
+        const float y = bf16_bits_value(a) * inv;  // the kernel's FP32 multiply
+        ok = ok && converter_e2m1(y) == exact_mag(a);
+      };
+      probe(0);
+      probe(0x7F7Fu);
+      for (int j = 0; j < 7; ++j) {
+        const uint32_t thr = t->code_thr[c][j];
+        if (thr <= 0x7F7Fu) {
+          probe(thr);
+          if (thr > 0) probe(thr - 1);
+        }
+      }
+      return ok;
     };
-    probe(0);
-    probe(0x7F7Fu);
-    for (int j = 0; j < 7; ++j) {
-      const uint32_t thr = t->code_thr[c][j];
-      if (thr <= 0x7F7Fu) {
-        probe(thr);
-        if (thr > 0) probe(thr - 1);
+    const float inv0 = t->inv[c];
+    const float up1 = nextafterf(inv0, INFINITY), dn1 = nextafterf(inv0, 0.0f);
+    const float cand[5] = {inv0, up1, dn1, nextafterf(up1, INFINITY), nextafterf(dn1, 0.0f)};
+    for (float inv : cand) {
+      if (passes(inv)) {
+        t->inv[c] = inv;
+        t->fast_ok[c >> 5] |= 1u << (c & 31);
+        break;
       }
     }
-    if (ok) t->fast_ok[c >> 5] |= 1u << (c & 31);
   }
 }
 
@@ -299,14 +315,15 @@ __device__ __forceinline__ void store_scale(const QuantParams& p, uint32_t sc, b
 // Streaming layout of the quantizer: one producer warp moves units of at most
 // 8192 BF16 elements (R rows x kc columns, 16 KB) from HBM into a ring of
 // shared-memory stages with bulk asynchronous copies; eight consumer warps
-// quantize each unit from shared memory, one 16-element block per thread per
-// pass.  Two CTAs per SM keep ~190 KB of loads in flight per SM.
-constexpr int kQConsumerWarps = 8;
+// quantize each unit from shared memory, one 16-element block per thread.
+// Two CTAs per SM keep ~190 KB of loads in flight per SM.
+constexpr int kQConsumerWarps = 16;
 constexpr int kQThreads = 32 * (kQConsumerWarps + 1);
 constexpr int kQStages = 6;
 constexpr int kQUnitElems = 8192;
 constexpr int kQUnitBytes = 2 * kQUnitElems;
 constexpr int kQSmem = kQStages * kQUnitBytes + 2 * 8 * kQStages + 64;
+static_assert(kQUnitElems / 16 == 32 * kQConsumerWarps, "one block per consumer thread per unit");
 
 __device__ unsigned int g_quant_error = 0;
 
@@ -384,7 +401,8 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
       uint32_t ph = 0;
       for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
         if (!q_wait(empty_bar(st), ph ^ 1u, abort_flag)) break;
-        const int64_t rb = u / p.col_units, cb = u % p.col_units;
+        const int64_t rb = p.col_units == 1 ? u : u / p.col_units;
+        const int64_t cb = p.col_units == 1 ? 0 : u % p.col_units;
         const int64_t r0 = rb * p.R;
         const int64_t rows = min(p.R, p.M - r0);
         const uint32_t row_bytes = (uint32_t)(p.kc * 2);
@@ -415,38 +433,30 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
       for (int i = 0; i < kQStages; ++i) q_wait(full_bar(i), (i < st) ? ph : (ph ^ 1u), abort_flag);
     }
   } else {
-    // ===== consumers =====
-    const int ctid = threadIdx.x;  // 0 .. 255
+    // ===== consumers: thread t quantizes block t of every unit =====
+    const int ctid = threadIdx.x;  // 0 .. 511
     const int64_t ublocks = p.R * p.nbu;  // blocks in a full unit
+    const int r = ctid / p.nbu, sb = ctid % p.nbu;  // the same place in every unit
+    const bool in_unit = ctid < ublocks;
+    const uint8_t* my_block = qsmem + 32 * ctid;
     int st = 0;
     uint32_t ph = 0;
     for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
       if (!q_wait(full_bar(st), ph, abort_flag)) break;
-      const int64_t rb = u / p.col_units, cb = u % p.col_units;
-      const int64_t r0 = rb * p.R;
-      const uint8_t* unit = qsmem + st * kQUnitBytes;
-      // This thread's blocks i = ctid, ctid + 256, ...: (row r, block sb) inside the unit.
-      int r = ctid / p.nbu, sb = ctid % p.nbu;
-      for (int64_t i0 = 0; i0 < ublocks; i0 += 32 * kQConsumerWarps) {
-        const int64_t i = i0 + ctid;
-        const int64_t m = r0 + r;
-        const int64_t sg = cb * p.nbu + sb;  // block index within the row
-        const bool valid = (i < ublocks) && (m < p.M);
-        uint32_t sc = 0;
-        if (valid) {
-          const uint4 q0 = *reinterpret_cast<const uint4*>(unit + 32 * i);
-          const uint4 q1 = *reinterpret_cast<const uint4*>(unit + 32 * i + 16);
-          const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-          sc = quantize_block(tab, p, w, m, sg, clips);
-        }
-        store_scale<kTiled, kGather4>(p, sc, valid, lane, m, sg, nb, katoms);
-        r += p.step_rows;
-        sb += p.step_blocks;
-        if (sb >= p.nbu) {
-          sb -= p.nbu;
-          ++r;
-        }
+      const int64_t rb = p.col_units == 1 ? u : u / p.col_units;
+      const int64_t cb = p.col_units == 1 ? 0 : u % p.col_units;
+      const int64_t m = rb * p.R + r;
+      const int64_t sg = cb * p.nbu + sb;  // block index within the row
+      const bool valid = in_unit && (m < p.M);
+      uint32_t sc = 0;
+      if (valid) {
+        const uint8_t* blk = my_block + st * kQUnitBytes;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(blk);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(blk + 16);
+        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        sc = quantize_block(tab, p, w, m, sg, clips);
       }
+      store_scale<kTiled, kGather4>(p, sc, valid, lane, m, sg, nb, katoms);
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
       if (++st == kQStages) {
