@@ -36,7 +36,20 @@ WORKLOAD = {"name": "qkv", "M": 32768, "K": 2688, "N": 8064}
 FP4_OVER_BF16 = 4.0        # nominal dense ratio 9 / 2.25 PFLOP/s
 QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16.0
 CPU_SAMPLE_ROWS = 64
+# DRAM bytes (read + write) of one GEMM launch on this workload, from an ncu
+# capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
+# kernel source it was taken on (first 16 hex digits of its SHA-256).
+GEMM_TRAFFIC = {"bytes": 536023552, "source_sha256": "3719e30700956cfb"}
 REF_ROWS = 16
+
+
+def gemm_traffic():
+    """Per-launch DRAM traffic of the GEMM if the kernel source is the one it was measured on."""
+    import hashlib
+    path = os.path.join(ROOT, "nvfp4_quantized_linear_fh_b200", "csrc", "fh_gemm.cu")
+    with open(path, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    return GEMM_TRAFFIC["bytes"] if digest == GEMM_TRAFFIC["source_sha256"] else None
 
 
 def peaks():
@@ -230,9 +243,8 @@ def bench_fh(args, rank, world, local_rank):
         t_e2e = e0.elapsed_time(e1) * 1e-3
 
     if world > 1:
-        t = torch.tensor([t_step, t_e2e, max(t_gemm), max(t_quant)], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_step, t_e2e = float(t[0]), float(t[1])
+        from nvfp4_quantized_linear_fh_b200 import dist as fhd
+        t_step, t_e2e = fhd.max_over_ranks([t_step, t_e2e], device=dev)
     flops = 2.0 * M * N * K
     return dict(t_step=t_step, t_quant=t_quant, t_gemm=t_gemm, t_e2e=t_e2e, e_steps=e_steps, flops=flops,
                 clips=clips, sampler=sampler.summary(), M=M, N=N, K=K,
@@ -241,6 +253,11 @@ def bench_fh(args, rank, world, local_rank):
 
 
 _WQ_CACHE = {}
+
+
+def gemm_bytes(M, N, K):
+    """Algorithmic bytes of one GEMM launch: A and W codes and scales, bias, BF16 output."""
+    return M * K // 2 + M * K // 16 + N * K // 2 + N * K // 16 + 2 * N + 2 * M * N
 
 
 def cpu_baseline(x_bits, w_bits, b_bits, sg_a, sg_w, rows):
@@ -342,7 +359,10 @@ def main():
         "roofline": {"kernel": "nvfp4_linear_kernel", "bound": "tensor", "achieved": achieved,
                      "peak": fp4_sust, "unit": "TFLOP/s", "frac": achieved / fp4_sust,
                      "peak_note": f"{pk['source']} bf16 sustained {pk['bf16_sustained']} x 4 (nominal FP4/BF16)",
-                     "frac_of_burst_peak": achieved / fp4_burst, "traffic": None},
+                     "frac_of_burst_peak": achieved / fp4_burst,
+                     "traffic": gemm_traffic() if r["M"] == WORKLOAD["M"] else None,
+                     "traffic_note": "bytes per launch, ncu dram__bytes_read.sum + dram__bytes_write.sum",
+                     "algorithmic_bytes": gemm_bytes(r["M"], r["N"], r["K"])},
         "quantizer": {"kernel": "quantize_kernel", "bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"],
                       "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"], "us": quant_mean * 1e6},
         "gemm_us": gemm_mean * 1e6, "clip_count": r["clips"],

@@ -145,6 +145,15 @@ int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64
  * x_dev and y_dev 16-byte aligned; in-place (x_dev == y_dev) is allowed. */
 int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t stream);
 
+/* Diagnostic of the failure path: enqueues a one-thread kernel whose bounded
+ * mbarrier wait (the same wait every pipeline stage of fh_nvfp4_linear uses)
+ * can never be satisfied and gives up after limit_us microseconds (1 .. 2e6),
+ * setting the device error word.  A following fh_device_status returns
+ * FH_ERR_TIMEOUT and the CUDA context stays usable.  The pages describe no
+ * failure handling; this exists so the timeout path can be tested without
+ * hanging or faulting a GPU. */
+int fh_selftest_bounded_wait(uint32_t limit_us, fh_stream_t stream);
+
 /* Synchronizes `stream`, then reads and clears the device error word of the
  * current device.  Returns FH_OK, FH_ERR_TIMEOUT if a kernel gave up on a
  * bounded wait since the last call, or FH_ERR_CUDA. */

@@ -58,6 +58,7 @@ _SIG = {
     "fh_scales_to_rowmajor": (_c.c_int, [_P, _P, _I64, _I64, _P]),
     "fh_gelu_bf16": (_c.c_int, [_P, _P, _I64, _P]),
     "fh_device_status": (_c.c_int, [_P]),
+    "fh_selftest_bounded_wait": (_c.c_int, [_c.c_uint32, _P]),
 }
 for _name, (_res, _args) in _SIG.items():
     _f = getattr(_lib, _name)
@@ -187,6 +188,11 @@ def fh_gelu_bf16(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
     if x.numel() != y.numel() or not x.is_contiguous() or not y.is_contiguous():
         raise ValueError("x and y must be contiguous with the same number of elements")
     _check(_lib.fh_gelu_bf16(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+
+
+def fh_selftest_bounded_wait(limit_us: int, stream=None) -> None:
+    """Enqueue the bounded-wait self-test (see include/fh.h); fh_device_status then reports the timeout."""
+    _check(_lib.fh_selftest_bounded_wait(int(limit_us), _stream(stream)))
 
 
 def fh_device_status(stream=None) -> None:

@@ -180,6 +180,15 @@ int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t 
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_gelu_bf16 launch");
 }
 
+int fh_selftest_bounded_wait(uint32_t limit_us, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (limit_us == 0 || limit_us > 2000000u)
+    return fail(FH_ERR_INVALID_ARG, "fh_selftest_bounded_wait: limit must be 1 us .. 2 s%s");
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_bounded_wait_selftest((uint64_t)limit_us * 1000u, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_selftest_bounded_wait launch");
+}
+
 int fh_device_status(fh_stream_t stream) {
   g_last_error[0] = 0;
   if (int st = check_device()) return st;

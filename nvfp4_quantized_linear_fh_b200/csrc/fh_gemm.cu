@@ -166,14 +166,15 @@ __device__ __forceinline__ uint64_t global_ns() {
 // when another role of the CTA already gave up), setting the device error word
 // and the CTA's abort flag.
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort,
+                                             uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t i = 1; i < (1u << 30); ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 255u) == 0u) {
       if (*abort) return false;
-      if (global_ns() - t0 > kWaitLimitNs) break;
+      if (global_ns() - t0 > limit_ns) break;
     }
   }
   atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
@@ -740,6 +741,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// arrives on, gives up after limit_ns, and sets the device error word.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(smem_u32(&bar), 1);
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  wait_bounded(smem_u32(&bar), 0, &abort_flag, limit_ns);
+}
+
 // ---- host side ----------------------------------------------------------------
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -834,6 +847,11 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
 }
 
 }  // namespace
+
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t s) {
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns);
+  return cudaGetLastError();
+}
 
 cudaError_t read_and_clear_device_error(unsigned int* bits, cudaStream_t s) {
   cudaError_t e = cudaStreamSynchronize(s);

@@ -33,6 +33,9 @@ cudaError_t launch_scales_to_rowmajor(const uint8_t* tiled, uint8_t* rowmajor, i
                                       int64_t K, cudaStream_t s);
 cudaError_t launch_gelu(const uint16_t* x, uint16_t* y, int64_t n, cudaStream_t s);
 
+// One-thread kernel whose bounded wait runs out after limit_ns (fh_gemm.cu).
+cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t s);
+
 // GEMM launcher (fh_gemm.cu).  Returns a CUDA error, or cudaErrorNotSupported
 // when the tensor maps cannot be built (message in *why).
 cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,

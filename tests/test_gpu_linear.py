@@ -151,3 +151,20 @@ def test_single_cta_form_matches_oracle():
                         "-k", "small or tiny or no_bias or back_to_back or full_size"],
                        env=env, capture_output=True, text=True, timeout=1200)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait that nothing satisfies gives up after its limit, the host reads
+    FH_ERR_TIMEOUT, and the next GEMM still runs correctly."""
+    m = fh()
+    m.fh_device_status()                      # clean start
+    m.fh_selftest_bounded_wait(200000)        # 0.2 s
+    with pytest.raises(m.FHError) as e:
+        m.fh_device_status()
+    assert e.value.status == m.FH_ERR_TIMEOUT
+    m.fh_device_status()                      # the word was cleared
+    x = S.random_bf16(("timeout", "x"), (130, 256), 1.0)
+    w = S.random_bf16(("timeout", "w"), (200, 256), 0.02)
+    y, _ = run_layer(x, w, None, 0.01, 0.0001)
+    check_linear(y, x, 0.01, w, 0.0001, None)
+    m.fh_device_status()
