@@ -128,7 +128,13 @@ int fh_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx,
  * Requires: M, N >= 0, K > 0, K % 64 == 0, N % 8 == 0, all pointers 16-byte
  * aligned, scales finite and > 0.  M == 0 or N == 0 enqueues nothing.
  * A bounded wait that expires inside the kernel sets the device error word
- * (see fh_device_status) instead of hanging. */
+ * (see fh_device_status) instead of hanging; the kernel then drains the
+ * copies and MMAs it issued and frees its TMEM before it exits.
+ * Environment: FH_GEMM_CTAS=1 (read at the first launch) selects the
+ * single-CTA form (128-row tiles) instead of the CTA pair;
+ * FH_GEMM_TEST_STALL=1 (read at each launch) is a test hook that makes the
+ * first CTA group's MMA warp stop after three stages of its first tile
+ * (K >= 1024), so the call ends with FH_ERR_TIMEOUT. */
 int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, float a_gscale,
                     const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
                     const uint16_t* bias_dev, uint16_t* y_dev, int64_t M, int64_t N,

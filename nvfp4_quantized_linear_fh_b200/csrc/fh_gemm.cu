@@ -115,6 +115,7 @@ struct Params {
   int sf_katoms;     // K / 64: 512-byte atoms per 128-row scale block
   int n_sfa_blocks;  // ceil(M / 128)
   int n_sfb_blocks;  // ceil(N / 128)
+  int stall_group;   // test hook: this CTA group's MMA warp stops after 3 stages (-1: none)
 };
 
 
@@ -180,6 +181,20 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
   atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
   *abort = 1;
   return false;
+}
+
+// Wait used while draining before exit: copies and MMAs this CTA issued must
+// have completed before it frees TMEM or retires, so this wait ignores the
+// abort flag and gives up only on its own time limit (~1 s).
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1; i < (1u << 30); ++i) {
+    if (mbar_try_wait(bar, parity)) return;
+    if ((i & 255u) == 0u && global_ns() - t0 > kDrainLimitNs) break;
+  }
+  atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
 }
 
 // Tensor TMA load into this CTA's shared memory.  kCta == 2: `bar` may be the
@@ -519,8 +534,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // of both CTAs land on its stage barriers).
       for (int s = 0; s < S; ++s) {
         const uint32_t par = (s < st.slot) ? st.phase : (st.phase ^ 1u);
-        wait_bounded(sfs_bar(s), par, abort_flag);
-        if (leader) wait_bounded(full_bar(s), par, abort_flag);
+        wait_drain(sfs_bar(s), par);
+        if (leader) wait_drain(full_bar(s), par);
       }
     }
   } else if (warp == 1) {
@@ -542,6 +557,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool landed = wait_bounded(full_bar(st.slot), st.phase, abort_flag) &&
                               wait_bounded(sff_bar(sf.slot), sf.phase, abort_flag);
           if (!__all_sync(0xFFFFFFFFu, landed)) {
+            ok = false;
+            break;
+          }
+          if (pair == p.stall_group && t == pair && kt == 3) {
+            // Test hook: stop issuing without committing, so every other role
+            // of this group runs into its bounded wait and takes the drain path.
             ok = false;
             break;
           }
@@ -584,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_commit_local2(drain_bar);
       }
       __syncwarp();
-      wait_bounded(drain_bar, 0, abort_flag);
+      wait_drain(drain_bar, 0);
     }
   } else if (warp >= kFirstSfWarp) {
     // ===================== scale stagers (every CTA) =====================
@@ -730,6 +751,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (kCta == 2 && *abort_flag != 0 && threadIdx.x == 0) {
+    // After a timeout the two producers may have stopped at different stages,
+    // and a peer's A/W copies complete on the leader's barriers, which this CTA
+    // cannot observe.  Give any such copy time to land before either CTA
+    // retires (copies take microseconds; this waits 2 ms).
+    const uint64_t t0 = global_ns();
+    while (global_ns() - t0 < 2000000ull) {
+    }
+  }
+  __syncthreads();
   if (kCta == 2) cluster_sync();  // the peer no longer needs this CTA's shared memory or TMEM
   tc_fence_after();
   if (warp == 1) {
@@ -783,6 +814,14 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uin
   return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Test hook: FH_GEMM_TEST_STALL=1 makes CTA group 0's MMA warp stop after three
+// stages of its first tile (when K spans at least four stages), so that the
+// kernel's bounded waits expire and the call ends with FH_ERR_TIMEOUT.
+int stall_group() {
+  const char* e = getenv("FH_GEMM_TEST_STALL");  // read per launch, so a test can switch it off again
+  return (e != nullptr && e[0] == '1') ? 0 : -1;
 }
 
 // Which kernel form to run: the CTA pair (default) or single CTAs.  The
@@ -896,6 +935,7 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
   p.sf_katoms = (int)(K / kMmaK);
   p.n_sfa_blocks = (int)((M + 127) / 128);
   p.n_sfb_blocks = (int)((N + 127) / 128);
+  p.stall_group = stall_group();
   return ctas == 2 ? launch_form<2>(tmA, tmB, tmY, p, s) : launch_form<1>(tmA, tmB, tmY, p, s);
 }
 

@@ -360,6 +360,24 @@ __device__ __forceinline__ bool q_wait(uint32_t bar, uint32_t parity, volatile i
   return false;
 }
 
+// Wait used by the producer's drain: its copies must have landed before the
+// CTA retires, so this ignores the abort flag and gives up only on its own
+// time limit (~1 s).
+__device__ __forceinline__ void q_wait_drain(uint32_t bar, uint32_t parity) {
+  if (q_try_wait(bar, parity)) return;
+  uint64_t t0;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t i = 1; i < (1u << 30); ++i) {
+    if (q_try_wait(bar, parity)) return;
+    if ((i & 255u) == 0u) {
+      uint64_t t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      if (t - t0 > 1000000000ull) break;
+    }
+  }
+  atomicOr(&g_quant_error, 1u);
+}
+
 // kGather4: K/16 % 4 == 0, so lanes 4i..4i+3 own four consecutive scales of
 // one row and store them as one word.
 template <bool kTiled, bool kGather4>
@@ -430,7 +448,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
         }
       }
       // Drain: every copy this thread issued has landed before the CTA retires.
-      for (int i = 0; i < kQStages; ++i) q_wait(full_bar(i), (i < st) ? ph : (ph ^ 1u), abort_flag);
+      for (int i = 0; i < kQStages; ++i) q_wait_drain(full_bar(i), (i < st) ? ph : (ph ^ 1u));
     }
   } else {
     // ===== consumers: thread t quantizes block t of every unit =====

@@ -168,3 +168,28 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     y, _ = run_layer(x, w, None, 0.01, 0.0001)
     check_linear(y, x, 0.01, w, 0.0001, None)
     m.fh_device_status()
+
+
+def test_gemm_stall_times_out_drains_and_context_survives(monkeypatch):
+    """With the test hook FH_GEMM_TEST_STALL=1 the first CTA pair's MMA warp
+    stops issuing after three stages of its first tile, without committing.
+    That pair's producer, scale stagers and epilogue then run into their
+    bounded waits (about 4 s) while copies and MMAs are in flight; the kernel
+    drains them and frees TMEM, and the host reads FH_ERR_TIMEOUT.  With the
+    hook off, the next GEMM in the same context passes parity."""
+    m = fh()
+    m.fh_device_status()                      # clean start
+    x = S.random_bf16(("stall", "x"), (1024, 2688), 1.0)
+    w = S.random_bf16(("stall", "w"), (1344, 2688), 0.02)
+    sg_a = oracle.scale_from_amax(oracle.amax(x))
+    sg_w = oracle.scale_from_amax(oracle.amax(w))
+    monkeypatch.setenv("FH_GEMM_TEST_STALL", "1")
+    run_layer(x, w, None, sg_a, sg_w)
+    monkeypatch.delenv("FH_GEMM_TEST_STALL")
+    with pytest.raises(m.FHError) as e:
+        m.fh_device_status()
+    assert e.value.status == m.FH_ERR_TIMEOUT
+    y, _ = run_layer(x, w, None, sg_a, sg_w)
+    rows = sample_rows(1024, 64, seed=5)
+    check_linear(y, x, sg_a, w, sg_w, None, rows=rows)
+    m.fh_device_status()
