@@ -39,7 +39,7 @@ CPU_SAMPLE_ROWS = 64
 # DRAM bytes (read + write) of one GEMM launch on this workload, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
 # kernel source it was taken on (first 16 hex digits of its SHA-256).
-GEMM_TRAFFIC = {"bytes": 535888128, "source_sha256": "fe5719c51338bdf4"}
+GEMM_TRAFFIC = {"bytes": 535854592, "source_sha256": "3d054c14f4714f94"}
 REF_ROWS = 16
 
 
@@ -91,7 +91,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "10"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except OSError:
@@ -111,7 +111,7 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         # samples taken while the timed region ran (nvidia-smi reports each sample
         # shortly after it is taken, so allow one interval of slack at the end)
@@ -124,6 +124,7 @@ class ClockSampler:
             try:
                 sm.append(float(parts[1]))
                 mx.append(float(parts[2]))
+                pw.append(float(parts[3]))
             except ValueError:
                 continue
             for n, v in zip(names, parts[5:9]):
@@ -132,7 +133,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm), "interval_ms": 20}
+                "power_w": statistics.median(pw) if pw else None, "samples": len(sm), "interval_ms": 10}
 
 
 def make_inputs(rank: int, M: int, quick: bool):
@@ -283,8 +284,10 @@ def cpu_baseline(x_bits, w_bits, b_bits, sg_a, sg_w, rows):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    # 250 steps of ~0.4 ms: a ~0.1 s timed region, long enough for the clock
+    # record to cover it and for the power limit to settle the clocks.
+    ap.add_argument("--steps", type=int, default=250)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="fh", choices=["fh", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--M", type=int, default=WORKLOAD["M"],
