@@ -803,19 +803,6 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
-                 uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Test hook: FH_GEMM_TEST_STALL=1 makes CTA group 0's MMA warp stop after three
 // stages of its first tile (when K spans at least four stages), so that the
 // kernel's bounded waits expire and the call ends with FH_ERR_TIMEOUT.
@@ -887,6 +874,19 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
 
 }  // namespace
 
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                        uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t s) {
   bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns);
   return cudaGetLastError();
@@ -909,12 +909,13 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
                                 cudaStream_t s, const char** why) {
   const int ctas = cta_mode();
   CUtensorMap tmA, tmB, tmY;
-  if (!make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2,
-                   BK / 2, 128) ||
-      !make_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
-                   BK / 2, BN / ctas) ||
-      !make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
-                   kEpiCols, 32)) {
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M,
+                          (uint64_t)K / 2, BK / 2, 128, sw) ||
+      !make_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N,
+                          (uint64_t)K / 2, BK / 2, BN / ctas, sw) ||
+      !make_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
+                          kEpiCols, 32, sw)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or a layout rule violated)";
     return cudaErrorNotSupported;
   }

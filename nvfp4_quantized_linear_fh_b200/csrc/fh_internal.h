@@ -1,6 +1,7 @@
 // fh_internal.h -- declarations shared by the CUDA translation units of libfh.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -21,6 +22,14 @@ cudaError_t read_and_clear_quant_error(unsigned int* bits);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// 2-D tiled tensor map of a row-major matrix (inner extent `inner` elements,
+// `outer` rows, rows `row_bytes` apart) with a box of box_inner x box_outer
+// elements; out-of-range elements of a box read as zero.  False if the driver
+// entry point is missing or a layout rule is violated (fh_gemm.cu).
+bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                        uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                        CUtensorMapSwizzle swizzle);
 
 // Quantizer / calibration / glue launchers (fh_quant.cu).  Arguments are
 // validated by the caller.

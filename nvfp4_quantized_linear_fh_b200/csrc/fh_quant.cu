@@ -27,10 +27,13 @@
 // threshold-compare path.  The block scale takes a converter candidate and
 // corrects it against the exact scale thresholds.
 //
-// Memory: each thread owns two 16-element blocks per step: two 32-byte loads,
-// two 8-byte code stores, and one 4-byte store of four consecutive block
-// scales per four lanes (gathered with shuffles).  HBM-bound: 2.5625 bytes per
-// element.
+// Memory: a producer warp streams 16 KB units of x into a ring of shared-memory
+// stages; each of 512 consumer threads quantizes one 16-element block per unit
+// (one 32-byte shared-memory read, one 8-byte code store; four lanes gather
+// four consecutive block scales into one 4-byte store).  For the tensor-core
+// scale layout a unit is a 128-row x 64-column tile, so each unit writes
+// exactly one 512-byte scale atom; for row-major scales a unit is whole rows.
+// HBM-bound: 2.5625 bytes per element.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -208,15 +211,6 @@ __device__ __forceinline__ uint32_t cvt_e4m3_sat(float v) {
   return r & 0xFFu;
 }
 
-// E2M1 x2 conversion: result bits 7..4 = code(hi), bits 3..0 = code(lo).
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float hi, float lo) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r)
-      : "f"(hi), "f"(lo));
-  return r;
-}
-
 // max(|a|, |b|) per BF16 half (sign bits = xor of the inputs' signs).
 __device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
   uint32_t r;
@@ -249,14 +243,33 @@ __device__ __noinline__ uint2 codes_exact(const QuantTable& t, uint32_t c, uint4
   return make_uint2(out[0], out[1]);
 }
 
+// Four BF16 words (8 values) -> 4 code bytes (low value in the low nibble);
+// the products x * inv are formed two at a time (mul.rn.f32x2: IEEE
+// round-to-nearest per lane, no flush to zero, the same as a scalar multiply).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float inv, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  uint32_t r;
+  asm("{\n\t.reg .b64 s, a0, a1, a2, a3;\n\t.reg .f32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t.reg .b8 t0, t1, t2, t3;\n\t"
+      "mov.b64 s, {%9, %9};\n\t"
+      "mov.b64 a0, {%1, %2};\n\tmov.b64 a1, {%3, %4};\n\tmov.b64 a2, {%5, %6};\n\tmov.b64 a3, {%7, %8};\n\t"
+      "mul.rn.f32x2 a0, a0, s;\n\tmul.rn.f32x2 a1, a1, s;\n\tmul.rn.f32x2 a2, a2, s;\n\tmul.rn.f32x2 a3, a3, s;\n\t"
+      "mov.b64 {l0, h0}, a0;\n\tmov.b64 {l1, h1}, a1;\n\tmov.b64 {l2, h2}, a2;\n\tmov.b64 {l3, h3}, a3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, h0, l0;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, h1, l1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t2, h2, l2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t3, h3, l3;\n\t"
+      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
+      : "=r"(r)
+      : "f"(__uint_as_float(w0 << 16)), "f"(__uint_as_float(w0 & 0xFFFF0000u)),
+        "f"(__uint_as_float(w1 << 16)), "f"(__uint_as_float(w1 & 0xFFFF0000u)),
+        "f"(__uint_as_float(w2 << 16)), "f"(__uint_as_float(w2 & 0xFFFF0000u)),
+        "f"(__uint_as_float(w3 << 16)), "f"(__uint_as_float(w3 & 0xFFFF0000u)), "f"(inv));
+  return r;
+}
+
 // 16 BF16 values -> 8 code bytes via the converter at multiplier inv.
 __device__ __forceinline__ void codes_fast(float inv, const uint32_t* w, uint32_t* out) {
-  uint32_t b[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    b[i] = cvt_e2m1x2(__uint_as_float(w[i] & 0xFFFF0000u) * inv, __uint_as_float(w[i] << 16) * inv);
-  out[0] = b[0] | (b[1] << 8) | (b[2] << 16) | (b[3] << 24);
-  out[1] = b[4] | (b[5] << 8) | (b[6] << 16) | (b[7] << 24);
+  out[0] = cvt_e2m1x8(inv, w[0], w[1], w[2], w[3]);
+  out[1] = cvt_e2m1x8(inv, w[4], w[5], w[6], w[7]);
 }
 
 __device__ __forceinline__ int64_t tiled_offset(int64_t m, int64_t s, int64_t katoms) {
@@ -312,11 +325,11 @@ __device__ __forceinline__ void store_scale(const QuantParams& p, uint32_t sc, b
   }
 }
 
-// Streaming layout of the quantizer: one producer warp moves units of at most
-// 8192 BF16 elements (R rows x kc columns, 16 KB) from HBM into a ring of
-// shared-memory stages with bulk asynchronous copies; eight consumer warps
-// quantize each unit from shared memory, one 16-element block per thread.
-// Two CTAs per SM keep ~190 KB of loads in flight per SM.
+// Streaming layout of the quantizer: one producer warp moves units of 8192 BF16
+// elements (16 KB) from HBM into a ring of shared-memory stages with
+// asynchronous bulk or tensor copies; sixteen consumer warps quantize each unit
+// from shared memory, one 16-element block per thread.  Two CTAs per SM keep
+// ~190 KB of loads in flight per SM.
 constexpr int kQConsumerWarps = 16;
 constexpr int kQThreads = 32 * (kQConsumerWarps + 1);
 constexpr int kQStages = 6;
@@ -378,9 +391,9 @@ __device__ __forceinline__ void q_wait_drain(uint32_t bar, uint32_t parity) {
   atomicOr(&g_quant_error, 1u);
 }
 
-// kGather4: K/16 % 4 == 0, so lanes 4i..4i+3 own four consecutive scales of
-// one row and store them as one word.
-template <bool kTiled, bool kGather4>
+// Row-major scale layout.  kGather4: K/16 % 4 == 0, so lanes 4i..4i+3 own four
+// consecutive scales of one row and store them as one word.
+template <bool kGather4>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(128) uint8_t qsmem[];
   __shared__ QuantTable tab;
@@ -474,7 +487,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
         const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
         sc = quantize_block(tab, p, w, m, sg, clips);
       }
-      store_scale<kTiled, kGather4>(p, sc, valid, lane, m, sg, nb, katoms);
+      store_scale<false, kGather4>(p, sc, valid, lane, m, sg, nb, katoms);
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
       if (++st == kQStages) {
@@ -484,15 +497,131 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
     }
   }
 
-  if (kTiled) {
-    // Zero the scales of the padding rows M .. ceil(M/128)*128 - 1.
-    const int64_t mpad = ((p.M + 127) >> 7) << 7;
-    const int64_t npad = (mpad - p.M) * nb;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += (int64_t)gridDim.x * blockDim.x)
-      p.scales[tiled_offset(p.M + i / nb, i % nb, katoms)] = 0;
+  // Clip count: warp sum, CTA sum, one atomic per CTA that saw any.
+  unsigned long long wsum = clips;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xFFFFFFFFu, wsum, o);
+  if (lane == 0 && wsum) atomicAdd(&cta_clips, wsum);
+  __syncthreads();
+  if (threadIdx.x == 0 && cta_clips && p.clip) atomicAdd(p.clip, cta_clips);
+}
+
+// Tensor-core scale layout: each unit is a 128-row x 64-column tile of x
+// (16 KB), loaded by one 2-D tensor TMA whose out-of-range rows read as zero.
+// Thread t quantizes block t % 4 of tile row t / 4, so one unit yields exactly
+// one 512-byte scale atom (written by the unit's own threads, which lets L2
+// merge it) and 32-byte code segments; zero rows past M give the zero padding
+// scales the layout requires.
+__global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_constant__ CUtensorMap tmx,
+                                                                   const __grid_constant__ QuantParams p) {
+  extern __shared__ __align__(128) uint8_t qsmem[];
+  __shared__ QuantTable tab;
+  __shared__ unsigned long long cta_clips;
+  __shared__ int abort_flag_s;
+  volatile int* abort_flag = &abort_flag_s;
+  const uint32_t stage0 = q_smem_u32(qsmem);
+  const uint32_t bar0 = stage0 + kQStages * kQUnitBytes;
+  auto full_bar = [&](int st) { return bar0 + 8u * st; };
+  auto empty_bar = [&](int st) { return bar0 + 8u * (kQStages + st); };
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(&p.tab);
+    uint4* dst = reinterpret_cast<uint4*>(&tab);
+    for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 16); i += blockDim.x) dst[i] = src[i];
+  }
+  if (threadIdx.x == 0) {
+    cta_clips = 0;
+    abort_flag_s = 0;
+    for (int st = 0; st < kQStages; ++st) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full_bar(st)));
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty_bar(st)), "r"(kQConsumerWarps));
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmx)) : "memory");
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t nb = p.K >> 4;
+  const int64_t katoms = nb >> 2;  // 64-column tiles per row block
+  unsigned long long clips = 0;
+  // Unit u is tile (u / katoms, u % katoms); the CTA visits u = blockIdx.x,
+  // blockIdx.x + gridDim.x, ..., so both coordinates advance by constants
+  // (no division inside the loops).
+  const int ka = (int)katoms;
+  const int d_row = (int)(gridDim.x / ka), d_col = (int)(gridDim.x % ka);
+  const int row0 = (int)(blockIdx.x / ka), col0 = (int)(blockIdx.x % ka);
+
+  if (warp == kQConsumerWarps) {
+    // ===== producer: one tensor TMA per 128 x 64 tile =====
+    if (lane == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      int tr = row0, tc = col0;
+      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+        if (!q_wait(empty_bar(st), ph ^ 1u, abort_flag)) break;
+        const int x0 = tc * 64, y0 = tr * 128;
+        tr += d_row;
+        tc += d_col;
+        if (tc >= ka) {
+          tc -= ka;
+          ++tr;
+        }
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full_bar(st)),
+                     "r"((uint32_t)kQUnitBytes)
+                     : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];" ::"r"(stage0 + st * kQUnitBytes),
+            "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(x0), "r"(y0), "r"(full_bar(st))
+            : "memory");
+        if (++st == kQStages) {
+          st = 0;
+          ph ^= 1u;
+        }
+      }
+      for (int i = 0; i < kQStages; ++i) q_wait_drain(full_bar(i), (i < st) ? ph : (ph ^ 1u));
+    }
+  } else {
+    // ===== consumers: thread t quantizes block t % 4 of tile row t / 4 =====
+    const int ctid = threadIdx.x;  // 0 .. 511
+    const int r = ctid >> 2, j = ctid & 3;
+    const uint8_t* my_block = qsmem + 32 * ctid;
+    int st = 0;
+    uint32_t ph = 0;
+    int tr = row0, tc = col0;
+    for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+      if (!q_wait(full_bar(st), ph, abort_flag)) break;
+      const int64_t m = (int64_t)tr * 128 + r;
+      const int64_t sg = (int64_t)tc * 4 + j;
+      tr += d_row;
+      tc += d_col;
+      if (tc >= ka) {
+        tc -= ka;
+        ++tr;
+      }
+      uint32_t sc = 0;
+      if (m < p.M) {
+        const uint8_t* blk = my_block + st * kQUnitBytes;
+        const uint4 q0 = *reinterpret_cast<const uint4*>(blk);
+        const uint4 q1 = *reinterpret_cast<const uint4*>(blk + 16);
+        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        sc = quantize_block(tab, p, w, m, sg, clips);
+      }
+      // Every row of the unit, padding rows included, writes its scales: the
+      // unit's atom starts at byte 512 u; lanes 4i..4i+3 (blocks 0..3 of row
+      // r) gather one word at r0 * 16 + r1 * 4 (r = r0 + 32 r1).
+      const uint32_t pair = sc | (__shfl_down_sync(0xFFFFFFFFu, sc, 1) << 8);
+      const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
+      if (j == 0) *reinterpret_cast<uint32_t*>(p.scales + u * 512 + (r & 31) * 16 + (r >> 5) * 4) = word;
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
+      if (++st == kQStages) {
+        st = 0;
+        ph ^= 1u;
+      }
+    }
   }
 
-  // Clip count: warp sum, CTA sum, one atomic per CTA that saw any.
   unsigned long long wsum = clips;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xFFFFFFFFu, wsum, o);
@@ -644,10 +773,28 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
     kernel<<<grid, kQThreads, kQSmem, s>>>(p);
     return cudaGetLastError();
   };
-  static int cfg_tt = -1, cfg_tf = -1, cfg_ft = -1, cfg_ff = -1;
-  if (tiled)
-    return gather4 ? launch(quantize_kernel<true, true>, cfg_tt) : launch(quantize_kernel<true, false>, cfg_tf);
-  return gather4 ? launch(quantize_kernel<false, true>, cfg_ft) : launch(quantize_kernel<false, false>, cfg_ff);
+  static int cfg_ft = -1, cfg_ff = -1;
+  if (tiled) {
+    // K % 64 == 0 here.  One unit per 128-row x 64-column tile.
+    CUtensorMap tmx;
+    if (!make_tensor_map_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M,
+                            (uint64_t)ldx * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorNotSupported;
+    p.n_units = ((M + 127) / 128) * (K / 64);
+    const int64_t tw = p.n_units > 0 ? p.n_units : 1;
+    const int tgrid = (int)(tw < 2 * (int64_t)sm_count() ? tw : 2 * (int64_t)sm_count());
+    static int cfg_t = -1;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cfg_t != dev) {
+      cudaError_t e = cudaFuncSetAttribute(quantize_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+      if (e != cudaSuccess) return e;
+      cfg_t = dev;
+    }
+    quantize_tiled_kernel<<<tgrid, kQThreads, kQSmem, s>>>(tmx, p);
+    return cudaGetLastError();
+  }
+  return gather4 ? launch(quantize_kernel<true>, cfg_ft) : launch(quantize_kernel<false>, cfg_ff);
 }
 
 cudaError_t read_and_clear_quant_error(unsigned int* bits) {
