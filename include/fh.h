@@ -140,6 +140,29 @@ int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, flo
                     const uint16_t* bias_dev, uint16_t* y_dev, int64_t M, int64_t N,
                     int64_t K, fh_stream_t stream);
 
+/* The NVFP4 linear layer fused with the activation that follows it and with
+ * the quantization of the next layer's input: the FFN's up projection, whose
+ * output feeds the down projection (FastH3 thread digest, tweet 5/8: the
+ * transformer's linear layers run in NVFP4; tweet 6/8: each FP4 layer's input
+ * is quantized with its calibrated scale).  For every output element,
+ *   y = bf16( a_gscale * w_gscale * sum_k A[m,k] * W[n,k] + bias[n] )
+ *   g = bf16( y/2 * erfc(-y / sqrt 2) )        (exact-erf GELU in FP32)
+ * exactly as fh_nvfp4_linear followed by fh_gelu_bf16 would compute them, and
+ * g is quantized with the next layer's global scale out_gscale exactly as
+ * fh_quantize_act does (FH_SCALES_MMA_TILED layout):
+ *   out_codes  [M, N/2], out_scales FH_SCALES_MMA_TILED of [M, N] (padding
+ *   rows zero), *out_clip_count_dev += elements with |g| > 2688 * out_gscale
+ *   (out_clip_count_dev may be NULL).
+ * y and g never reach memory: the BF16 intermediate of M * N * 2 bytes is not
+ * written or read.  The outputs are bit-identical to the three separate calls.
+ * Requires everything fh_nvfp4_linear requires, N % 64 == 0, out_gscale finite
+ * and > 0, out_codes_dev and out_scales_dev 16-byte aligned. */
+int fh_nvfp4_linear_gelu_quant(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, float a_gscale,
+                               const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                               const uint16_t* bias_dev, float out_gscale, uint8_t* out_codes_dev,
+                               uint8_t* out_scales_dev, unsigned long long* out_clip_count_dev,
+                               int64_t M, int64_t N, int64_t K, fh_stream_t stream);
+
 /* Permute FH_SCALES_MMA_TILED scales of a [rows, K] matrix into row-major
  * [rows, K/16] (drops the padding).  Requires K % 64 == 0. */
 int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows,

@@ -55,6 +55,8 @@ _SIG = {
     "fh_amax": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P]),
     "fh_quantize_act": (_c.c_int, [_P, _I64, _I64, _I64, _c.c_float, _P, _P, _P, _c.c_int, _P]),
     "fh_nvfp4_linear": (_c.c_int, [_P, _P, _c.c_float, _P, _P, _c.c_float, _P, _P, _I64, _I64, _I64, _P]),
+    "fh_nvfp4_linear_gelu_quant": (_c.c_int, [_P, _P, _c.c_float, _P, _P, _c.c_float, _P, _c.c_float, _P, _P, _P,
+                                              _I64, _I64, _I64, _P]),
     "fh_scales_to_rowmajor": (_c.c_int, [_P, _P, _I64, _I64, _P]),
     "fh_gelu_bf16": (_c.c_int, [_P, _P, _I64, _P]),
     "fh_device_status": (_c.c_int, [_P]),
@@ -172,6 +174,38 @@ def fh_nvfp4_linear(a_codes: torch.Tensor, a_scales: torch.Tensor, a_gscale: flo
             raise ValueError("bias must be contiguous with N elements")
     _check(_lib.fh_nvfp4_linear(_ptr(a_codes), _ptr(a_scales), float(a_gscale), _ptr(w_codes), _ptr(w_scales),
                                 float(w_gscale), _ptr(bias), _ptr(y), M, N, K, _stream(stream)))
+
+
+def fh_nvfp4_linear_gelu_quant(a_codes: torch.Tensor, a_scales: torch.Tensor, a_gscale: float,
+                               w_codes: torch.Tensor, w_scales: torch.Tensor, w_gscale: float,
+                               bias: torch.Tensor | None, out_gscale: float, out_codes: torch.Tensor,
+                               out_scales: torch.Tensor, out_clip: torch.Tensor | None = None, stream=None) -> None:
+    """NVFP4 input of the next layer, GELU(bf16(a_g * w_g * A . W^T + bias)) quantized with out_gscale,
+    written as out_codes [M, N/2] and tensor-core-layout out_scales; out_clip (int64, 1 element) += clips."""
+    for t, n in ((a_codes, "a_codes"), (w_codes, "w_codes"), (out_codes, "out_codes")):
+        _need(t, _U8, n, 2)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(a_scales, _U8, "a_scales")
+    _need(w_scales, _U8, "w_scales")
+    _need(out_scales, _U8, "out_scales")
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K or tuple(out_codes.shape) != (M, N // 2):
+        raise ValueError("shape mismatch: a_codes [M, K/2], w_codes [N, K/2], out_codes [M, N/2]")
+    if (a_scales.numel() < fh_scales_bytes(M, K) or w_scales.numel() < fh_scales_bytes(N, K)
+            or out_scales.numel() < fh_scales_bytes(M, N)):
+        raise ValueError("scale arrays too small for the tensor-core scale layout")
+    if bias is not None:
+        _need(bias, _BF16, "bias")
+        if bias.numel() != N or not bias.is_contiguous():
+            raise ValueError("bias must be contiguous with N elements")
+    if out_clip is not None and (out_clip.dtype != torch.int64 or out_clip.device.type != "cuda"):
+        raise TypeError("out_clip must be a CUDA int64 tensor")
+    _check(_lib.fh_nvfp4_linear_gelu_quant(_ptr(a_codes), _ptr(a_scales), float(a_gscale), _ptr(w_codes),
+                                           _ptr(w_scales), float(w_gscale), _ptr(bias), float(out_gscale),
+                                           _ptr(out_codes), _ptr(out_scales), _ptr(out_clip), M, N, K,
+                                           _stream(stream)))
 
 
 def fh_scales_to_rowmajor(tiled: torch.Tensor, rowmajor: torch.Tensor, rows: int, K: int, stream=None) -> None:

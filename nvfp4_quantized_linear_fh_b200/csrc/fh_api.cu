@@ -155,6 +155,37 @@ int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, flo
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear launch");
 }
 
+int fh_nvfp4_linear_gelu_quant(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, float a_gscale,
+                               const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                               const uint16_t* bias_dev, float out_gscale, uint8_t* out_codes_dev,
+                               uint8_t* out_scales_dev, unsigned long long* out_clip_count_dev,
+                               int64_t M, int64_t N, int64_t K, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!(a_gscale > 0.0f) || isinf(a_gscale) || !(w_gscale > 0.0f) || isinf(w_gscale) || !(out_gscale > 0.0f) ||
+      isinf(out_gscale))
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_gelu_quant: global scales must be finite and > 0%s");
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || N % 64 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_nvfp4_linear_gelu_quant: need M, N >= 0, K > 0, K %% 64 == 0, N %% 64 == 0%s");
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_gelu_quant: each dimension must fit in 31 bits%s");
+  if (M == 0 || N == 0) return FH_OK;
+  if (a_codes_dev == nullptr || a_scales_dev == nullptr || w_codes_dev == nullptr || w_scales_dev == nullptr ||
+      out_codes_dev == nullptr || out_scales_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_gelu_quant: null pointer%s");
+  if (!aligned16(a_codes_dev) || !aligned16(a_scales_dev) || !aligned16(w_codes_dev) || !aligned16(w_scales_dev) ||
+      !aligned16(out_codes_dev) || !aligned16(out_scales_dev) || (bias_dev != nullptr && !aligned16(bias_dev)))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_gelu_quant: every pointer must be 16-byte aligned%s");
+  if (int st = check_device()) return st;
+  const char* why = nullptr;
+  cudaError_t e = fh::launch_nvfp4_linear_gelu_quant(a_codes_dev, a_scales_dev, a_gscale, w_codes_dev, w_scales_dev,
+                                                     w_gscale, bias_dev, out_gscale, out_codes_dev, out_scales_dev,
+                                                     out_clip_count_dev, M, N, K, (cudaStream_t)stream, &why);
+  if (e == cudaErrorNotSupported && why != nullptr)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_gelu_quant: %s", why);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear_gelu_quant launch");
+}
+
 int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows, int64_t K,
                           fh_stream_t stream) {
   g_last_error[0] = 0;

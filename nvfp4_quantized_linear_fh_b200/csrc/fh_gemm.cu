@@ -45,6 +45,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include "fh_internal.h"
 
@@ -116,6 +117,30 @@ struct Params {
   int n_sfa_blocks;  // ceil(M / 128)
   int n_sfb_blocks;  // ceil(N / 128)
   int stall_group;   // test hook: this CTA group's MMA warp stops after 3 stages (-1: none)
+};
+
+// Epilogue mode 1: instead of y, emit the next layer's NVFP4 input
+// g = GELU(bf16(alpha * acc + bias)) quantized with that layer's global scale:
+// codes [M, N/2] and tensor-core-layout scales of [M, N] (N % 64 == 0), plus
+// the count of clipped elements of g.
+struct EpiQuant {
+  QuantTable tab;  // decision table of the next layer's global scale
+  uint8_t* codes;
+  uint8_t* scales;
+  unsigned long long* clip;  // may be null
+  float inv6sg;
+  uint32_t clip_thr;
+  int katoms;  // N / 64: scale atoms per 128-row block
+  int m_pad;   // rows of the scale array: ceil(M / 128) * 128
+};
+struct EpiNone {};
+template <int kEpi>
+struct EpiSel {
+  using type = EpiNone;
+};
+template <>
+struct EpiSel<1> {
+  using type = EpiQuant;
 };
 
 
@@ -422,10 +447,11 @@ struct Ring {
   }
 };
 
-template <int kCta>
+template <int kCta, int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmY, const Params p) {
+                        const __grid_constant__ CUtensorMap tmY, const Params p,
+                        const __grid_constant__ typename EpiSel<kEpi>::type eq) {
   using C = Cfg<kCta>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -442,6 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto sfe_bar = [&](int b) { return bar0 + 8u * (3 * S + 4 + kSfBufs + b); };  // each CTA: scale buffer free
   const uint32_t drain_bar = bar0 + 8u * (3 * S + 4 + 2 * kSfBufs);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kNumBars * 8);
+  if constexpr (kEpi == 1) {
+    // The next layer's decision table, in the (otherwise unused) output staging area.
+    static_assert(sizeof(QuantTable) <= kEpiWarps * C::kEpiBufs * kEpiBufBytes, "table fits the staging area");
+    const uint4* src = reinterpret_cast<const uint4*>(&eq.tab);
+    uint4* dst = reinterpret_cast<uint4*>(smem + C::kOffEpi);
+    for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 16); i += blockDim.x) dst[i] = src[i];
+  }
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + C::kNumBars * 8 + 8);
 
   const int warp = threadIdx.x >> 5;
@@ -673,6 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     int buf = 0;
+    unsigned long long clips = 0;  // kEpi == 1: clipped elements of g in this thread's rows
     for (int t = pair; t < p.num_tiles; t += npairs) {
       const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
       const int row0 = m_tile * C::BM + (int)rank * 128 + 32 * q;  // this warp's 32 output rows
@@ -714,6 +748,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           packed[2 * j] = pack_bf16x2(y0, y1);
           packed[2 * j + 1] = pack_bf16x2(y2, y3);
         }
+        if constexpr (kEpi == 1) {
+          // g = GELU(y) per element, then four 16-column blocks of row `row`.
+          const QuantTable& qt = *reinterpret_cast<const QuantTable*>(smem + C::kOffEpi);
+          const int row = row0 + lane;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            packed[i] = nvfp4::gelu_bits(packed[i] & 0xFFFFu) | (nvfp4::gelu_bits(packed[i] >> 16) << 16);
+          uint32_t word = 0;
+          uint2 cd[4];
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            uint32_t amax;
+            const uint32_t sc = nvfp4::quantize_block_codes(qt, eq.inv6sg, packed + 8 * b, amax, cd[b]);
+            word |= sc << (8 * b);
+            if (row < p.M) clips += nvfp4::block_clips(packed + 8 * b, amax, eq.clip_thr);
+          }
+          if (row < p.M) {
+            uint4* dst = reinterpret_cast<uint4*>(eq.codes + (size_t)row * (size_t)(p.N >> 1) + (col0 >> 1));
+            dst[0] = make_uint4(cd[0].x, cd[0].y, cd[1].x, cd[1].y);
+            dst[1] = make_uint4(cd[2].x, cd[2].y, cd[3].x, cd[3].y);
+          }
+          // Scale atom (row / 128, col0 / 64); rows M .. m_pad - 1 get zero scales.
+          if (row < eq.m_pad)
+            *reinterpret_cast<uint32_t*>(eq.scales + ((size_t)(row >> 7) * eq.katoms + (col0 >> 6)) * 512 +
+                                         (row & 31) * 16 + ((row >> 5) & 3) * 4) = row < p.M ? word : 0u;
+          continue;
+        }
         // Reuse a staging buffer only after its previous TMA store has read it.
         if (lane == 0) {
           if (C::kEpiBufs == 1)
@@ -746,6 +807,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (lane == 0) bulk_wait_all();
+    if constexpr (kEpi == 1) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) clips += __shfl_xor_sync(0xFFFFFFFFu, clips, o);
+      if (lane == 0 && clips != 0 && eq.clip != nullptr) atomicAdd(eq.clip, clips);
+    }
     __syncwarp();
   }
 
@@ -823,9 +889,9 @@ int cta_mode() {
   return mode;
 }
 
-template <int kCta>
+template <int kCta, int kEpi>
 cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const Params& p,
-                        cudaStream_t s) {
+                        const typename EpiSel<kEpi>::type& eq, cudaStream_t s) {
   using C = Cfg<kCta>;
   static int configured_device = -1;
   static int max_groups = 0;
@@ -833,7 +899,7 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
   cudaGetDevice(&dev);
   if (configured_device != dev) {
     cudaError_t e =
-        cudaFuncSetAttribute(nvfp4_linear_kernel<kCta>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+        cudaFuncSetAttribute(nvfp4_linear_kernel<kCta, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
     if (e != cudaSuccess) return e;
     max_groups = sm_count() / kCta;
     if (kCta == 2) {
@@ -850,7 +916,7 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4_linear_kernel<2>, &cfg) == cudaSuccess && clusters > 0)
+      if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4_linear_kernel<2, kEpi>, &cfg) == cudaSuccess && clusters > 0)
         max_groups = clusters < max_groups ? clusters : max_groups;
       cudaGetLastError();
     }
@@ -869,7 +935,7 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = kCta == 2 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta>, tmA, tmB, tmY, p);
+  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi>, tmA, tmB, tmY, p, eq);
 }
 
 }  // namespace
@@ -903,10 +969,13 @@ cudaError_t read_and_clear_device_error(unsigned int* bits, cudaStream_t s) {
   return e;
 }
 
-cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,
-                                const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
-                                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
-                                cudaStream_t s, const char** why) {
+namespace {
+
+// Shared by both epilogue modes: tensor maps, tile counts and the launch.
+// y is the BF16 output (mode 0) or null (mode 1, outputs in *eq).
+cudaError_t launch_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g, const uint8_t* w_codes,
+                          const uint8_t* w_scales, float w_g, const uint16_t* bias, uint16_t* y, int64_t M,
+                          int64_t N, int64_t K, const EpiQuant* eq, cudaStream_t s, const char** why) {
   const int ctas = cta_mode();
   CUtensorMap tmA, tmB, tmY;
   const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
@@ -914,11 +983,12 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
                           (uint64_t)K / 2, BK / 2, 128, sw) ||
       !make_tensor_map_2d(&tmB, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_codes, (uint64_t)K / 2, (uint64_t)N,
                           (uint64_t)K / 2, BK / 2, BN / ctas, sw) ||
-      !make_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M, (uint64_t)N * 2,
-                          kEpiCols, 32, sw)) {
+      (y != nullptr && !make_tensor_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, y, (uint64_t)N, (uint64_t)M,
+                                           (uint64_t)N * 2, kEpiCols, 32, sw))) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or a layout rule violated)";
     return cudaErrorNotSupported;
   }
+  if (y == nullptr) tmY = tmA;  // unused by the quantizing epilogue
   Params p;
   p.sfa = a_scales;
   p.sfb = w_scales;
@@ -937,7 +1007,37 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
   p.n_sfa_blocks = (int)((M + 127) / 128);
   p.n_sfb_blocks = (int)((N + 127) / 128);
   p.stall_group = stall_group();
-  return ctas == 2 ? launch_form<2>(tmA, tmB, tmY, p, s) : launch_form<1>(tmA, tmB, tmY, p, s);
+  if (eq == nullptr) {
+    const EpiNone none;
+    return ctas == 2 ? launch_form<2, 0>(tmA, tmB, tmY, p, none, s) : launch_form<1, 0>(tmA, tmB, tmY, p, none, s);
+  }
+  return ctas == 2 ? launch_form<2, 1>(tmA, tmB, tmY, p, *eq, s) : launch_form<1, 1>(tmA, tmB, tmY, p, *eq, s);
+}
+
+}  // namespace
+
+cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,
+                                const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
+                                const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                                cudaStream_t s, const char** why) {
+  return launch_linear(a_codes, a_scales, a_g, w_codes, w_scales, w_g, bias, y, M, N, K, nullptr, s, why);
+}
+
+cudaError_t launch_nvfp4_linear_gelu_quant(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,
+                                           const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
+                                           const uint16_t* bias, float out_g, uint8_t* out_codes,
+                                           uint8_t* out_scales, unsigned long long* out_clip, int64_t M,
+                                           int64_t N, int64_t K, cudaStream_t s, const char** why) {
+  static thread_local EpiQuant eq;  // 2.9 KB: kept off the stack
+  memcpy(&eq.tab, &quant_table_for(out_g), sizeof(QuantTable));
+  eq.codes = out_codes;
+  eq.scales = out_scales;
+  eq.clip = out_clip;
+  eq.inv6sg = (float)(1.0 / (6.0 * (double)out_g));
+  eq.clip_thr = clip_threshold_bits(out_g);
+  eq.katoms = (int)(N / 64);
+  eq.m_pad = (int)(((M + 127) / 128) * 128);
+  return launch_linear(a_codes, a_scales, a_g, w_codes, w_scales, w_g, bias, nullptr, M, N, K, &eq, s, why);
 }
 
 }  // namespace fh

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "../../include/fh.h"
+#include "fh_nvfp4.cuh"
 
 namespace fh {
 
@@ -31,6 +32,12 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
                         uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                         CUtensorMapSwizzle swizzle);
 
+// Exact decision table of the NVFP4 quantizer for global scale sg (host, cached
+// per thread), and the BF16 bits of the smallest magnitude strictly beyond
+// 2688 sg (the clip threshold) (fh_quant.cu).
+const QuantTable& quant_table_for(float sg);
+uint32_t clip_threshold_bits(float sg);
+
 // Quantizer / calibration / glue launchers (fh_quant.cu).  Arguments are
 // validated by the caller.
 cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float sg,
@@ -51,5 +58,15 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
                                 const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
                                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N,
                                 int64_t K, cudaStream_t s, const char** why);
+
+// The same GEMM with the epilogue that emits the next layer's NVFP4 input:
+// GELU(bf16(alpha * acc + bias)) quantized with global scale out_g into
+// out_codes [M, N/2] and tensor-core-layout out_scales of [M, N]; clipped
+// elements are added to *out_clip (if not null).  Requires N % 64 == 0.
+cudaError_t launch_nvfp4_linear_gelu_quant(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,
+                                           const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
+                                           const uint16_t* bias, float out_g, uint8_t* out_codes,
+                                           uint8_t* out_scales, unsigned long long* out_clip, int64_t M,
+                                           int64_t N, int64_t K, cudaStream_t s, const char** why);
 
 }  // namespace fh

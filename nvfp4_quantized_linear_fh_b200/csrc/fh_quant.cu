@@ -40,6 +40,7 @@
 #include <string.h>
 
 #include "fh_internal.h"
+#include "fh_nvfp4.cuh"
 
 namespace fh {
 
@@ -47,13 +48,7 @@ namespace {
 
 constexpr uint32_t kBf16Inf = 0x7F80u;
 
-struct __align__(16) QuantTable {
-  uint16_t code_thr[128][8];  // [c][j<7]: smallest |x| (BF16 bits) whose exact magnitude code is >= j+1 at scale code c
-  uint16_t scale_thr[128];    // [c]: smallest block amax (BF16 bits) whose exact scale code is >= c
-  float inv[128];             // 1 / (S_c * s_g): multiplier of the converter path (0 for c == 0)
-  uint32_t fast_ok[4];        // bit c: the converter path is exact at scale code c
-};
-static_assert(sizeof(QuantTable) % 16 == 0, "table copy granularity");
+using namespace nvfp4;
 
 struct QuantParams {
   QuantTable tab;
@@ -183,8 +178,10 @@ void build_table(float sg_f, QuantTable* t) {
   }
 }
 
+}  // namespace
+
 // Small per-thread cache: calibrated layers reuse one s_g for every call.
-const QuantTable& table_for(float sg) {
+const QuantTable& quant_table_for(float sg) {
   struct Entry {
     float sg;
     bool valid;
@@ -202,75 +199,11 @@ const QuantTable& table_for(float sg) {
   return e.t;
 }
 
+uint32_t clip_threshold_bits(float sg) { return bf16_threshold(2688.0 * (double)sg, true); }
+
+namespace {
+
 // ---- device --------------------------------------------------------------------
-
-// E4M3 x2 conversion (round to nearest even, saturating); the low byte's code.
-__device__ __forceinline__ uint32_t cvt_e4m3_sat(float v) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
-  return r & 0xFFu;
-}
-
-// max(|a|, |b|) per BF16 half (sign bits = xor of the inputs' signs).
-__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-__device__ __forceinline__ float bf16_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
-
-// 16 BF16 values (words w0..w7 in q0, q1) -> 8 code bytes, exact-threshold path.
-// Out of line: only blocks whose scale code failed the converter check get here.
-__device__ __noinline__ uint2 codes_exact(const QuantTable& t, uint32_t c, uint4 q0, uint4 q1) {
-  const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-  uint32_t thr[7];
-#pragma unroll
-  for (int j = 0; j < 7; ++j) thr[j] = t.code_thr[c][j];
-  uint32_t out[2] = {0, 0};
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const uint32_t lo = w[i] & 0xFFFFu, hi = w[i] >> 16;
-    uint32_t ml = 0, mh = 0;
-#pragma unroll
-    for (int j = 0; j < 7; ++j) {
-      ml += ((lo & 0x7FFFu) >= thr[j]) ? 1u : 0u;
-      mh += ((hi & 0x7FFFu) >= thr[j]) ? 1u : 0u;
-    }
-    const uint32_t byte = (ml | ((lo >> 12) & 8u)) | ((mh | ((hi >> 12) & 8u)) << 4);
-    out[i >> 2] |= byte << (8 * (i & 3));
-  }
-  return make_uint2(out[0], out[1]);
-}
-
-// Four BF16 words (8 values) -> 4 code bytes (low value in the low nibble);
-// the products x * inv are formed two at a time (mul.rn.f32x2: IEEE
-// round-to-nearest per lane, no flush to zero, the same as a scalar multiply).
-__device__ __forceinline__ uint32_t cvt_e2m1x8(float inv, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
-  uint32_t r;
-  asm("{\n\t.reg .b64 s, a0, a1, a2, a3;\n\t.reg .f32 l0, h0, l1, h1, l2, h2, l3, h3;\n\t.reg .b8 t0, t1, t2, t3;\n\t"
-      "mov.b64 s, {%9, %9};\n\t"
-      "mov.b64 a0, {%1, %2};\n\tmov.b64 a1, {%3, %4};\n\tmov.b64 a2, {%5, %6};\n\tmov.b64 a3, {%7, %8};\n\t"
-      "mul.rn.f32x2 a0, a0, s;\n\tmul.rn.f32x2 a1, a1, s;\n\tmul.rn.f32x2 a2, a2, s;\n\tmul.rn.f32x2 a3, a3, s;\n\t"
-      "mov.b64 {l0, h0}, a0;\n\tmov.b64 {l1, h1}, a1;\n\tmov.b64 {l2, h2}, a2;\n\tmov.b64 {l3, h3}, a3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t0, h0, l0;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t1, h1, l1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t2, h2, l2;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t3, h3, l3;\n\t"
-      "mov.b32 %0, {t0, t1, t2, t3};\n\t}"
-      : "=r"(r)
-      : "f"(__uint_as_float(w0 << 16)), "f"(__uint_as_float(w0 & 0xFFFF0000u)),
-        "f"(__uint_as_float(w1 << 16)), "f"(__uint_as_float(w1 & 0xFFFF0000u)),
-        "f"(__uint_as_float(w2 << 16)), "f"(__uint_as_float(w2 & 0xFFFF0000u)),
-        "f"(__uint_as_float(w3 << 16)), "f"(__uint_as_float(w3 & 0xFFFF0000u)), "f"(inv));
-  return r;
-}
-
-// 16 BF16 values -> 8 code bytes via the converter at multiplier inv.
-__device__ __forceinline__ void codes_fast(float inv, const uint32_t* w, uint32_t* out) {
-  out[0] = cvt_e2m1x8(inv, w[0], w[1], w[2], w[3]);
-  out[1] = cvt_e2m1x8(inv, w[4], w[5], w[6], w[7]);
-}
 
 __device__ __forceinline__ int64_t tiled_offset(int64_t m, int64_t s, int64_t katoms) {
   return ((m >> 7) * katoms + (s >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (s & 3);
@@ -281,33 +214,11 @@ __device__ __forceinline__ int64_t tiled_offset(int64_t m, int64_t s, int64_t ka
 __device__ __forceinline__ uint32_t quantize_block(const QuantTable& tab, const QuantParams& p,
                                                    const uint32_t* w, int64_t m, int64_t s,
                                                    unsigned long long& clips) {
-  // Block amax over the magnitudes (a max, so exact).
-  const uint32_t r01 = max_abs_bf16x2(w[0], w[1]), r23 = max_abs_bf16x2(w[2], w[3]);
-  const uint32_t r45 = max_abs_bf16x2(w[4], w[5]), r67 = max_abs_bf16x2(w[6], w[7]);
-  const uint32_t r = max_abs_bf16x2(max_abs_bf16x2(r01, r23), max_abs_bf16x2(r45, r67));
-  const uint32_t amax = max_abs_bf16x2(r, __byte_perm(r, 0, 0x1032)) & 0x7FFFu;
-  // Scale code: converter candidate, corrected against the exact thresholds.
-  const float amax_f = bf16_to_float(amax);
-  uint32_t c = min(cvt_e4m3_sat(amax_f * p.inv6sg), 126u);
-  while (c < 126u && amax >= tab.scale_thr[c + 1]) ++c;
-  while (c > 0u && amax < tab.scale_thr[c]) --c;
+  uint32_t amax;
   uint2 out;
-  const float inv = tab.inv[c];
-  if (((tab.fast_ok[c >> 5] >> (c & 31)) & 1u) && (amax_f * inv <= 3.0e38f)) {
-    uint32_t o[2];
-    codes_fast(inv, w, o);
-    out = make_uint2(o[0], o[1]);
-  } else {
-    out = codes_exact(tab, c, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));
-  }
+  const uint32_t c = quantize_block_codes(tab, p.inv6sg, w, amax, out);
   *reinterpret_cast<uint2*>(p.codes + m * (p.K >> 1) + 8 * s) = out;
-  if (amax >= p.clip_thr) {  // only blocks reaching beyond the limit hold clipped elements
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      clips += ((w[i] & 0x7FFFu) >= p.clip_thr) ? 1u : 0u;
-      clips += (((w[i] >> 16) & 0x7FFFu) >= p.clip_thr) ? 1u : 0u;
-    }
-  }
+  clips += block_clips(w, amax, p.clip_thr);
   return c;
 }
 
@@ -690,14 +601,6 @@ __global__ void scales_to_rowmajor_kernel(const uint8_t* __restrict__ tiled,
   }
 }
 
-__device__ __forceinline__ uint32_t gelu_bits(uint32_t bits16) {
-  const float v = bf16_to_float(bits16);
-  // x/2 * erfc(-x/sqrt 2) == x/2 * (1 + erf(x/sqrt 2)), without the cancellation
-  // of 1 + erf for negative x.
-  const float y = 0.5f * v * erfcf(-v * 0.70710678118654752440f);
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y));
-}
-
 __global__ void gelu_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict__ y, int64_t n) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t nvec = n >> 3;
@@ -724,7 +627,7 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
                             uint8_t* codes, uint8_t* scales, unsigned long long* clip,
                             int layout, cudaStream_t s) {
   QuantParams p;
-  memcpy(&p.tab, &table_for(sg), sizeof(QuantTable));
+  memcpy(&p.tab, &quant_table_for(sg), sizeof(QuantTable));
   p.x = x;
   p.codes = codes;
   p.scales = scales;
@@ -757,7 +660,7 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   }
   // Exact clip threshold: smallest BF16 magnitude strictly beyond 2688 * s_g
   // (2688 * s_g is exact in FP64: 5 + 24 significant bits).
-  p.clip_thr = bf16_threshold(2688.0 * (double)sg, true);
+  p.clip_thr = clip_threshold_bits(sg);
   const bool tiled = layout == FH_SCALES_MMA_TILED;
   const bool gather4 = (K / 16) % 4 == 0;
   const int64_t want = p.n_units > 0 ? p.n_units : 1;

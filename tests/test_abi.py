@@ -96,6 +96,16 @@ def test_argument_validation_without_gpu(lib):
     assert g(None, fake, 1.0, fake, fake, 1.0, None, fake, 128, 256, 128, None) == 1
     assert g(fake, fake, 1.0, fake, fake, 1.0, None, fake, 0, 256, 128, None) == 0    # empty
     assert g(fake, fake, 1.0, fake, fake, 1.0, None, fake, 128, 0, 128, None) == 0
+    f = lib.fh_nvfp4_linear_gelu_quant
+    f.argtypes = [P, P, ctypes.c_float, P, P, ctypes.c_float, P, ctypes.c_float, P, P, P,
+                  ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P]
+    assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, fake, fake, None, 128, 200, 128, None) == 2  # N % 64
+    assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, fake, fake, None, 128, 256, 96, None) == 2   # K % 64
+    assert f(fake, fake, 1.0, fake, fake, 1.0, None, 0.0, fake, fake, None, 128, 256, 128, None) == 1  # out scale
+    assert f(fake, fake, 1.0, fake, fake, 1.0, None, float("inf"), fake, fake, None, 128, 256, 128, None) == 1
+    assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, None, fake, None, 128, 256, 128, None) == 1  # null codes
+    assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, P(24), fake, None, 128, 256, 128, None) == 2
+    assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, fake, fake, None, 0, 256, 128, None) == 0   # empty
     a = lib.fh_amax
     a.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P]
     assert a(fake, 3, 5, 4, fake, None) == 2
