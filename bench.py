@@ -281,6 +281,108 @@ def cpu_baseline(x_bits, w_bits, b_bits, sg_a, sg_w, rows):
     return 2.0 * rows * N * K / dt / 1e12, dt, cores
 
 
+def bench_ffn(args):
+    """The FFN block of the 2688-wide transformer (up 2688->10752, GELU, down
+    10752->2688) on args.M tokens, timed two ways on the same operands:
+    unfused (quantize, GEMM, GELU, quantize, GEMM) and fused (quantize, GEMM
+    whose epilogue applies GELU and quantizes for the down projection, GEMM)."""
+    import torch
+    import synthetic as S
+    import nvfp4_quantized_linear_fh_b200 as fh
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    up, down = S.workloads()["ffn"]
+    M, K, N1 = args.M, up.K, up.N
+    N2 = down.N
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    def quant_weight(layer):
+        w = to_dev(S.weights(layer))
+        wamax = torch.zeros(1, dtype=torch.float32, device=dev)
+        fh.fh_amax(w, wamax)
+        sg = fh.fh_scale_from_amax(wamax.item())
+        wc, wsc = fh.empty_quantized(layer.N, layer.K, device=dev)
+        fh.fh_quantize_act(w, sg, wc, wsc, None)
+        return wc, wsc, sg, to_dev(S.bias(layer))
+
+    import dataclasses
+    x = to_dev(S.activations(dataclasses.replace(up, M=M, n_calib=max(up.n_calib, M // up.batch))))
+    w1c, w1s, sg_w1, b1 = quant_weight(up)
+    w2c, w2s, sg_w2, b2 = quant_weight(down)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    fh.fh_amax(x, amax)
+    sg_x = fh.fh_scale_from_amax(amax.item())
+    xc, xs = fh.empty_quantized(M, K, device=dev)
+    y1 = torch.empty((M, N1), dtype=torch.bfloat16, device=dev)
+    g = torch.empty_like(y1)
+    gc, gs = fh.empty_quantized(M, N1, device=dev)
+    out = torch.empty((M, N2), dtype=torch.bfloat16, device=dev)
+    # Down-projection input scale: calibrated on the GELU output of this input.
+    fh.fh_quantize_act(x, sg_x, xc, xs, None)
+    fh.fh_nvfp4_linear(xc, xs, sg_x, w1c, w1s, sg_w1, b1, y1)
+    fh.fh_gelu_bf16(y1, g)
+    amax.zero_()
+    fh.fh_amax(g, amax)
+    sg_g = fh.fh_scale_from_amax(amax.item())
+
+    def unfused():
+        fh.fh_quantize_act(x, sg_x, xc, xs, None)
+        fh.fh_nvfp4_linear(xc, xs, sg_x, w1c, w1s, sg_w1, b1, y1)
+        fh.fh_gelu_bf16(y1, g)
+        fh.fh_quantize_act(g, sg_g, gc, gs, None)
+        fh.fh_nvfp4_linear(gc, gs, sg_g, w2c, w2s, sg_w2, b2, out)
+
+    def gelu_quant():
+        fh.fh_quantize_act(x, sg_x, xc, xs, None)
+        fh.fh_nvfp4_linear(xc, xs, sg_x, w1c, w1s, sg_w1, b1, y1)
+        fh.fh_gelu_quantize_act(y1, sg_g, gc, gs, None)
+        fh.fh_nvfp4_linear(gc, gs, sg_g, w2c, w2s, sg_w2, b2, out)
+
+    def fused():
+        fh.fh_quantize_act(x, sg_x, xc, xs, None)
+        fh.fh_nvfp4_linear_gelu_quant(xc, xs, sg_x, w1c, w1s, sg_w1, b1, sg_g, gc, gs, None)
+        fh.fh_nvfp4_linear(gc, gs, sg_g, w2c, w2s, sg_w2, b2, out)
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) * 1e-3 / steps
+
+    steps = max(1, min(args.steps, 100))
+    variants = {"unfused": (unfused, "quantize, linear, gelu, quantize, linear"),
+                "gelu_quant": (gelu_quant, "quantize, linear, gelu_quantize, linear"),
+                "fused_epilogue": (fused, "quantize, linear_gelu_quant, linear")}
+    times, identical, ref_out = {}, True, None
+    for name, (fn, _) in variants.items():
+        times[name] = timed(fn, steps)
+        if ref_out is None:
+            ref_out = out.clone()
+        else:
+            identical = identical and bool(torch.equal(out.view(torch.int16), ref_out.view(torch.int16)))
+    fh.fh_device_status()
+    flops = 2.0 * M * K * N1 + 2.0 * M * N1 * N2
+    best = min(times, key=times.get)
+    print(json.dumps({
+        "metric": "NVFP4 FFN block TFLOPS (up 2688->10752, GELU, down 10752->2688)", "unit": "TFLOPS",
+        "value": flops / times[best] / 1e12, "ms_per_step": times[best] * 1e3, "best": best, "steps": steps,
+        "warmup": args.warmup, "n_gpus": 1, "higher_is_better": True,
+        "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": f"FFN block {M}x2688->10752->2688 per GPU", "M": M},
+        "variants": {n: {"value": flops / t / 1e12, "ms_per_step": t * 1e3, "calls": variants[n][1]}
+                     for n, t in times.items()},
+        "outputs_bit_identical": identical}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -293,10 +395,15 @@ def main():
     ap.add_argument("--M", type=int, default=WORKLOAD["M"],
                     help="token rows per GPU (profiling cases use fewer than the workload's 32768)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--workload", default="qkv", choices=["qkv", "ffn"],
+                    help="qkv: the headline line (fused QKV layer); ffn: the FFN block, fused vs unfused epilogue")
     ap.add_argument("--quick", action="store_true",
                     help="calibrate on the input batches only (setup shortcut for profiling cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.workload == "ffn":
+        bench_ffn(args)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

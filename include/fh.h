@@ -115,6 +115,17 @@ int fh_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx,
                     unsigned long long* clip_count_dev, int scale_layout,
                     fh_stream_t stream);
 
+/* NVFP4 quantization of GELU(x) for BF16 x [M, K] (leading dimension ldx):
+ * the FFN's activation applied while quantizing the down projection's input,
+ * so GELU(x) is never written.  Bit-identical to fh_gelu_bf16 followed by
+ * fh_quantize_act with FH_SCALES_MMA_TILED (same GELU arithmetic, same
+ * rounding rules); outputs and clip count as for fh_quantize_act.  Requires
+ * K % 64 == 0, ldx >= K, ldx % 8 == 0, 16-byte aligned pointers, s_g finite
+ * and > 0. */
+int fh_gelu_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx, float global_scale,
+                         uint8_t* codes_dev, uint8_t* scales_dev, unsigned long long* clip_count_dev,
+                         fh_stream_t stream);
+
 /* NVFP4 linear layer on the tcgen05 tensor cores (FastH3 thread digest, tweet
  * 5/8: the transformer's linear layers in NVFP4 on Blackwell):
  *   y[m, n] = bf16( a_gscale * w_gscale * sum_k A[m,k] * W[n,k] + bias[n] )
@@ -169,9 +180,11 @@ int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64
                           int64_t K, fh_stream_t stream);
 
 /* Exact-erf GELU on BF16, y = bf16(x/2 * (1 + erf(x/sqrt 2))), evaluated in
- * FP32 as x/2 * erfc(-x/sqrt 2) (no cancellation for negative x); the
- * activation between the two linear layers of the FFN.  n >= 0;
- * x_dev and y_dev 16-byte aligned; in-place (x_dev == y_dev) is allowed. */
+ * FP32 as x/2 * erfc(-x/sqrt 2) (no cancellation for negative x), with erfc
+ * from a Chebyshev-fitted approximation of fractional error below 1.2e-7 (far
+ * below BF16's 2^-8); the activation between the two linear layers of the
+ * FFN.  n >= 0; x_dev and y_dev 16-byte aligned; in-place (x_dev == y_dev)
+ * is allowed. */
 int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t stream);
 
 /* Diagnostic of the failure path: enqueues a one-thread kernel whose bounded

@@ -54,6 +54,7 @@ _SIG = {
     "fh_scales_bytes": (_c.c_size_t, [_I64, _I64, _c.c_int]),
     "fh_amax": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P]),
     "fh_quantize_act": (_c.c_int, [_P, _I64, _I64, _I64, _c.c_float, _P, _P, _P, _c.c_int, _P]),
+    "fh_gelu_quantize_act": (_c.c_int, [_P, _I64, _I64, _I64, _c.c_float, _P, _P, _P, _P]),
     "fh_nvfp4_linear": (_c.c_int, [_P, _P, _c.c_float, _P, _P, _c.c_float, _P, _P, _I64, _I64, _I64, _P]),
     "fh_nvfp4_linear_gelu_quant": (_c.c_int, [_P, _P, _c.c_float, _P, _P, _c.c_float, _P, _c.c_float, _P, _P, _P,
                                               _I64, _I64, _I64, _P]),
@@ -149,6 +150,25 @@ def fh_quantize_act(x: torch.Tensor, global_scale: float, codes: torch.Tensor, s
         _need(clip_count, (torch.int64, torch.uint64), "clip_count")
     _check(_lib.fh_quantize_act(_ptr(x), M, K, x.stride(0), float(global_scale), _ptr(codes), _ptr(scales),
                                 _ptr(clip_count), scale_layout, _stream(stream)))
+
+
+def fh_gelu_quantize_act(x: torch.Tensor, global_scale: float, codes: torch.Tensor, scales: torch.Tensor,
+                         clip_count: torch.Tensor | None = None, stream=None) -> None:
+    """NVFP4 codes and tensor-core-layout scales of GELU(x) for BF16 x [M, K] (row stride x.stride(0))."""
+    _need(x, _BF16, "x", 2)
+    if x.stride(1) != 1:
+        raise ValueError("x must be row-major (unit column stride)")
+    _need(codes, _U8, "codes", 2)
+    _need(scales, _U8, "scales")
+    M, K = x.shape
+    if tuple(codes.shape) != (M, K // 2) or not codes.is_contiguous():
+        raise ValueError("codes must be a contiguous [M, K/2] uint8 tensor")
+    if scales.numel() < fh_scales_bytes(M, K):
+        raise ValueError("scales too small for the tensor-core scale layout")
+    if clip_count is not None and (clip_count.dtype != torch.int64 or clip_count.device.type != "cuda"):
+        raise TypeError("clip_count must be a CUDA int64 tensor")
+    _check(_lib.fh_gelu_quantize_act(_ptr(x), M, K, x.stride(0), float(global_scale), _ptr(codes), _ptr(scales),
+                                     _ptr(clip_count), _stream(stream)))
 
 
 def fh_nvfp4_linear(a_codes: torch.Tensor, a_scales: torch.Tensor, a_gscale: float,

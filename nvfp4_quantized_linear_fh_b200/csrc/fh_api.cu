@@ -125,8 +125,30 @@ int fh_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx, fl
     return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_quantize_act: tensor too large%s");
   if (int st = check_device()) return st;
   cudaError_t e = fh::launch_quantize(x_dev, M, K, ldx, global_scale, codes_dev, scales_dev, clip_count_dev,
-                                      scale_layout, (cudaStream_t)stream);
+                                      scale_layout, false, (cudaStream_t)stream);
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_quantize_act launch");
+}
+
+int fh_gelu_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx, float global_scale,
+                         uint8_t* codes_dev, uint8_t* scales_dev, unsigned long long* clip_count_dev,
+                         fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!(global_scale > 0.0f) || isinf(global_scale))
+    return fail(FH_ERR_INVALID_ARG, "fh_gelu_quantize_act: global scale must be finite and > 0%s");
+  if (M < 0 || K <= 0 || K % 64 != 0 || ldx < K || ldx % 8 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_gelu_quantize_act: need M >= 0, K > 0, K %% 64 == 0, ldx >= K, ldx %% 8 == 0%s");
+  if (M == 0) return FH_OK;
+  if (x_dev == nullptr || codes_dev == nullptr || scales_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_gelu_quantize_act: null pointer%s");
+  if (!aligned16(x_dev) || !aligned16(codes_dev) || !aligned16(scales_dev))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_gelu_quantize_act: x, codes and scales must be 16-byte aligned%s");
+  if (M * (K / 16) > ((int64_t)1 << 40))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_gelu_quantize_act: tensor too large%s");
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_quantize(x_dev, M, K, ldx, global_scale, codes_dev, scales_dev, clip_count_dev,
+                                      FH_SCALES_MMA_TILED, true, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_gelu_quantize_act launch");
 }
 
 int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, float a_gscale,

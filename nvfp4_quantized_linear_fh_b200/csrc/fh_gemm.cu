@@ -754,7 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int row = row0 + lane;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            packed[i] = nvfp4::gelu_bits(packed[i] & 0xFFFFu) | (nvfp4::gelu_bits(packed[i] >> 16) << 16);
+            packed[i] = nvfp4::gelu2_bits(packed[i]);
           uint32_t word = 0;
           uint2 cd[4];
 #pragma unroll

@@ -40,9 +40,10 @@ uint32_t clip_threshold_bits(float sg);
 
 // Quantizer / calibration / glue launchers (fh_quant.cu).  Arguments are
 // validated by the caller.
+// gelu: quantize GELU(x) (tensor-core scale layout only).
 cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float sg,
                             uint8_t* codes, uint8_t* scales, unsigned long long* clip,
-                            int layout, cudaStream_t s);
+                            int layout, bool gelu, cudaStream_t s);
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ldx, float* amax,
                         cudaStream_t s);
 cudaError_t launch_scales_to_rowmajor(const uint8_t* tiled, uint8_t* rowmajor, int64_t rows,

@@ -133,14 +133,56 @@ __device__ __forceinline__ uint32_t block_clips(const uint32_t* w, uint32_t amax
   return n;
 }
 
-// Exact-erf GELU of one BF16 value, rounded to BF16:
-// x/2 * erfc(-x/sqrt 2) == x/2 * (1 + erf(x/sqrt 2)), without the cancellation
-// of 1 + erf for negative x.
-__device__ __forceinline__ uint32_t gelu_bits(uint32_t bits16) {
-  const float v = bf16_to_float(bits16);
-  const float y = 0.5f * v * erfcf(-v * 0.70710678118654752440f);
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(y));
+// GELU of both BF16 halves of w (the low half is the first element), rounded
+// to BF16 and packed the same way:
+//   GELU(x) = x/2 * erfc(-x/sqrt 2) = x/2 * (1 + erf(x/sqrt 2)),
+// using erfc(-x/sqrt 2) = 2 - erfc(x/sqrt 2) for x >= 0, so there is no
+// 1 + erf cancellation for negative x.  erfc(z), z >= 0, takes the
+// Chebyshev-fitted form
+//   erfc(z) ~= t * exp(-z^2 + P(t)),  t = 1 / (1 + z/2),
+// with P of degree 9, whose fractional error is below 1.2e-7 for every z >= 0
+// (Press, Teukolsky, Vetterling and Flannery, Numerical Recipes, 2nd ed.,
+// section 6.2).  In FP32 with the hardware reciprocal and base-2 exponent the
+// relative error stays near 1e-6, far below BF16's 2^-8; values below the FP32
+// normal range flush to zero.  The two elements go through the packed FP32x2
+// pipe together.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
+
+__device__ __forceinline__ uint32_t gelu2_bits(uint32_t w) {
+  const float2 v = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  const float2 z = __fmul2_rn(make_float2(__uint_as_float((w << 16) & 0x7FFFFFFFu),
+                                          __uint_as_float(w & 0x7FFF0000u)),
+                              make_float2(0.70710678118654752440f, 0.70710678118654752440f));
+  const float2 d = __ffma2_rn(make_float2(0.5f, 0.5f), z, make_float2(1.0f, 1.0f));
+  const float2 t = make_float2(__fdividef(1.0f, d.x), __fdividef(1.0f, d.y));
+  float2 p = make_float2(0.17087277f, 0.17087277f);
+  p = __ffma2_rn(p, t, make_float2(-0.82215223f, -0.82215223f));
+  p = __ffma2_rn(p, t, make_float2(1.48851587f, 1.48851587f));
+  p = __ffma2_rn(p, t, make_float2(-1.13520398f, -1.13520398f));
+  p = __ffma2_rn(p, t, make_float2(0.27886807f, 0.27886807f));
+  p = __ffma2_rn(p, t, make_float2(-0.18628806f, -0.18628806f));
+  p = __ffma2_rn(p, t, make_float2(0.09678418f, 0.09678418f));
+  p = __ffma2_rn(p, t, make_float2(0.37409196f, 0.37409196f));
+  p = __ffma2_rn(p, t, make_float2(1.00002368f, 1.00002368f));
+  p = __ffma2_rn(p, t, make_float2(-1.26551223f, -1.26551223f));
+  // exp(-z^2 + P) = 2^((-z^2 + P) * log2(e))
+  const float2 a = __fmul2_rn(__ffma2_rn(make_float2(-z.x, -z.y), z, p),
+                              make_float2(1.44269504088896340736f, 1.44269504088896340736f));
+  const float2 e = __fmul2_rn(t, make_float2(ex2_approx(a.x), ex2_approx(a.y)));
+  const float2 phi2 = make_float2(v.x >= 0.0f ? 2.0f - e.x : e.x, v.y >= 0.0f ? 2.0f - e.y : e.y);
+  const float2 y = __fmul2_rn(__fmul2_rn(make_float2(0.5f, 0.5f), v), phi2);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(y.y), "f"(y.x));
+  return r;
+}
+
+// GELU of one BF16 value (low 16 bits), rounded to BF16: the same arithmetic
+// as gelu2_bits.
+__device__ __forceinline__ uint32_t gelu_bits(uint32_t bits16) { return gelu2_bits(bits16 & 0xFFFFu) & 0xFFFFu; }
 
 }  // namespace nvfp4
 }  // namespace fh

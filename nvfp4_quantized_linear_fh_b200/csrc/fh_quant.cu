@@ -423,6 +423,9 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
 // one 512-byte scale atom (written by the unit's own threads, which lets L2
 // merge it) and 32-byte code segments; zero rows past M give the zero padding
 // scales the layout requires.
+// kGelu: quantize GELU(x) instead of x (the FFN activation applied on the way,
+// with the same arithmetic as the stand-alone GELU kernel).
+template <bool kGelu>
 __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                    const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(128) uint8_t qsmem[];
@@ -515,7 +518,11 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
         const uint8_t* blk = my_block + st * kQUnitBytes;
         const uint4 q0 = *reinterpret_cast<const uint4*>(blk);
         const uint4 q1 = *reinterpret_cast<const uint4*>(blk + 16);
-        const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+        if (kGelu) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) w[i] = gelu2_bits(w[i]);
+        }
         sc = quantize_block(tab, p, w, m, sg, clips);
       }
       // Every row of the unit, padding rows included, writes its scales: the
@@ -608,7 +615,7 @@ __global__ void gelu_kernel(const uint16_t* __restrict__ x, uint16_t* __restrict
     uint4 v = reinterpret_cast<const uint4*>(x)[i];
     uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) w[k] = gelu_bits(w[k] & 0xFFFFu) | (gelu_bits(w[k] >> 16) << 16);
+    for (int k = 0; k < 4; ++k) w[k] = gelu2_bits(w[k]);
     reinterpret_cast<uint4*>(y)[i] = make_uint4(w[0], w[1], w[2], w[3]);
   }
   for (int64_t i = (nvec << 3) + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
@@ -625,7 +632,7 @@ int grid_for(int64_t work_items, int threads, int per_sm) {
 
 cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float sg,
                             uint8_t* codes, uint8_t* scales, unsigned long long* clip,
-                            int layout, cudaStream_t s) {
+                            int layout, bool gelu, cudaStream_t s) {
   QuantParams p;
   memcpy(&p.tab, &quant_table_for(sg), sizeof(QuantTable));
   p.x = x;
@@ -686,15 +693,16 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
     p.n_units = ((M + 127) / 128) * (K / 64);
     const int64_t tw = p.n_units > 0 ? p.n_units : 1;
     const int tgrid = (int)(tw < 2 * (int64_t)sm_count() ? tw : 2 * (int64_t)sm_count());
-    static int cfg_t = -1;
+    static int cfg_t[2] = {-1, -1};
     int dev = 0;
     cudaGetDevice(&dev);
-    if (cfg_t != dev) {
-      cudaError_t e = cudaFuncSetAttribute(quantize_tiled_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
+    auto kernel = gelu ? quantize_tiled_kernel<true> : quantize_tiled_kernel<false>;
+    if (cfg_t[gelu] != dev) {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
       if (e != cudaSuccess) return e;
-      cfg_t = dev;
+      cfg_t[gelu] = dev;
     }
-    quantize_tiled_kernel<<<tgrid, kQThreads, kQSmem, s>>>(tmx, p);
+    kernel<<<tgrid, kQThreads, kQSmem, s>>>(tmx, p);
     return cudaGetLastError();
   }
   return gather4 ? launch(quantize_kernel<true>, cfg_ft) : launch(quantize_kernel<false>, cfg_ff);

@@ -132,3 +132,29 @@ def test_fused_single_cta_form():
                         "-k", "matches_three_calls or clip_counts"],
                        env=env, capture_output=True, text=True, timeout=1200)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+@pytest.mark.parametrize("M,K", [(100, 192), (129, 512), (300, 2688), (1, 64), (513, 10752)])
+def test_gelu_quantize_matches_two_calls(M, K):
+    """fh_gelu_quantize_act == fh_gelu_bf16 then fh_quantize_act, bit for bit
+    (codes, every scale byte including padding rows, clip count)."""
+    m = fh()
+    y = to_dev(S.random_bf16(("gq", M, K), (M, K), 2.0))
+    g = torch.empty_like(y)
+    m.fh_gelu_bf16(y, g)
+    torch.cuda.synchronize()
+    g_bits = g.view(torch.int16).cpu().numpy().view(np.uint16)
+    sg = oracle.scale_from_amax(oracle.amax(g_bits) * 0.5)
+    rc, rsc, rclip = quantize_tiled(g, sg)
+    oc, osc = m.empty_quantized(M, K)
+    oc.fill_(0xA5)
+    osc.fill_(0xA5)
+    oclip = torch.zeros(1, dtype=torch.int64, device="cuda")
+    m.fh_gelu_quantize_act(y, sg, oc, osc, oclip)
+    torch.cuda.synchronize()
+    m.fh_device_status()
+    _assert_identical(dict(ref=(rc, rsc, int(rclip.item())), got=(oc, osc, int(oclip.item()))))
+    if M * K <= 300 * 2688:  # and the oracle's quantization of the same GELU output
+        oc_, osc_, oclip_ = oracle.quantize(g_bits, sg)
+        np.testing.assert_array_equal(oc.cpu().numpy(), oc_)
+        assert int(oclip.item()) == oclip_
