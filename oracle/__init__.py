@@ -190,3 +190,43 @@ def gelu(x_bits: np.ndarray) -> np.ndarray:
     y = np.empty(x.size, dtype=np.float64)
     lib().oracle_gelu(_ptr(x), x.size, _ptr(y))
     return y.reshape(np.shape(x_bits))
+
+
+# ---- INT8 query/key quantization for attention scores ----------------------
+#
+# FastH3 Trim (comfyui-wiki news), "How fast it runs": on the RTX 4090 the
+# FP8 path quantizes the query and the key to INT8 for the score computation.
+# The pages fix neither the granularity nor the rounding; this oracle takes the
+# plainest reading: one symmetric scale per row (one token of one head),
+#   s = fp32(amax_row / 127)                      (IEEE single division)
+#   q = clamp(rne(fp32(x / s)), -127, 127)        (IEEE single division, then
+#                                                  round half to even)
+# with s = 0 and q = 0 for an all-zero row.  The decisions are taken in FP32
+# because the kernel takes them in FP32; numpy's float32 division is the IEEE
+# correctly rounded one.
+
+def quantize_int8_rows(x_bits: np.ndarray):
+    """BF16 bits [rows, d] -> (int8 [rows, d], float32 scales [rows])."""
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32).reshape(x_bits.shape)
+    amax = np.abs(x).max(axis=1).astype(np.float32)
+    s = (amax / np.float32(127.0)).astype(np.float32)
+    q = np.zeros(x.shape, dtype=np.int8)
+    nz = s > 0
+    with np.errstate(invalid="ignore", divide="ignore"):
+        r = (x[nz] / s[nz, None]).astype(np.float32)
+    q[nz] = np.clip(np.rint(r), -127, 127).astype(np.int8)
+    return q, s
+
+
+def int8_scores(q8: np.ndarray, q_scales: np.ndarray, k8: np.ndarray, k_scales: np.ndarray,
+                sm_scale: float) -> np.ndarray:
+    """S[h, i, j] = sm_scale * s_q[h, i] * s_k[h, j] * sum_d q[h, i, d] k[h, j, d] in binary64
+    (the integer sums are exact); q8 [H, Tq, d], k8 [H, Tk, d], scales [H, T]."""
+    acc = np.einsum("hid,hjd->hij", q8.astype(np.int64), k8.astype(np.int64))
+    return (float(sm_scale) * q_scales.astype(np.float64)[:, :, None] * k_scales.astype(np.float64)[:, None, :]
+            * acc.astype(np.float64))
+
+
+def int8_scores_tolerance(s_ref: np.ndarray) -> np.ndarray:
+    """Three FP32 roundings of an exact product: 2e-6 relative (2^-21 = 4.8e-7 each), plus 1e-30."""
+    return 2e-6 * np.abs(s_ref) + 1e-30
