@@ -25,8 +25,8 @@
  * Conventions for every entry point:
  *   - Pointers named *_dev or documented as device pointers are device memory
  *     owned by the caller; the library allocates nothing and keeps no state
- *     between calls except a per-device property cache and one device error
- *     word.
+ *     between calls except a per-device property cache and the device error
+ *     words that fh_device_status reads.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
  *     stream) and the call returns without synchronizing, except where stated.
  *   - The return value is an fh_status.  On failure nothing was enqueued and
@@ -186,6 +186,35 @@ int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64
  * FFN.  n >= 0; x_dev and y_dev 16-byte aligned; in-place (x_dev == y_dev)
  * is allowed. */
 int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t stream);
+
+/* INT8 query/key quantization for attention scores.  FastH3 Trim
+ * (comfyui-wiki news), "How fast it runs": where no FP4 tensor cores exist,
+ * the query and the key are quantized to INT8 for the score computation.  The
+ * pages fix neither the granularity nor the rounding; this library takes one
+ * symmetric scale per row (one token of one head), in IEEE FP32:
+ *   s = amax_row / 127,   q = clamp(round_half_even(x / s), -127, 127),
+ * with s = 0 and q = 0 for an all-zero row.
+ * x_dev: BF16 [rows, d], rows ldx elements apart; q_dev: int8 [rows, d], dense
+ * (rows d bytes apart); scales_dev: FP32 [rows].  rows >= 0, d > 0, d % 8 == 0,
+ * ldx >= d, ldx % 8 == 0; x_dev and q_dev 16-byte aligned, scales_dev 4-byte
+ * aligned.  Bit-exact: every decision is one IEEE single division. */
+int fh_quantize_int8_rows(const uint16_t* x_dev, int64_t rows, int64_t d, int64_t ldx, int8_t* q_dev,
+                          float* scales_dev, fh_stream_t stream);
+
+/* Attention scores from INT8 queries and keys (same passage as above):
+ *   S[h, i, j] = (float(acc) * (s_q[h, i] * sm_scale)) * s_k[h, j],
+ *   acc = sum_c q[h, i, c] * k[h, j, c]   (exact INT32 on the tensor cores),
+ * every product an FP32 multiply rounded to nearest.
+ * q_dev: int8 [heads, tq, d]; k_dev: int8 [heads, tk, d]; q_scales_dev FP32
+ * [heads, tq]; k_scales_dev FP32 [heads, tk] (the outputs of
+ * fh_quantize_int8_rows over the flattened rows); s_dev: FP32 [heads, tq, tk],
+ * every element written.  heads, tq, tk >= 0 (each below 2^31); d > 0,
+ * d % 16 == 0, d <= 65536; tk % 4 == 0; q_dev, k_dev and s_dev 16-byte
+ * aligned; sm_scale finite.  A bounded wait that expires sets the device error
+ * word (fh_device_status) and the kernel drains and returns. */
+int fh_int8_attention_scores(const int8_t* q_dev, const float* q_scales_dev, const int8_t* k_dev,
+                             const float* k_scales_dev, float sm_scale, float* s_dev, int64_t heads, int64_t tq,
+                             int64_t tk, int64_t d, fh_stream_t stream);
 
 /* Diagnostic of the failure path: enqueues a one-thread kernel whose bounded
  * mbarrier wait (the same wait every pipeline stage of fh_nvfp4_linear uses)

@@ -60,6 +60,8 @@ _SIG = {
                                               _I64, _I64, _I64, _P]),
     "fh_scales_to_rowmajor": (_c.c_int, [_P, _P, _I64, _I64, _P]),
     "fh_gelu_bf16": (_c.c_int, [_P, _P, _I64, _P]),
+    "fh_quantize_int8_rows": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "fh_int8_attention_scores": (_c.c_int, [_P, _P, _P, _P, _c.c_float, _P, _I64, _I64, _I64, _I64, _P]),
     "fh_device_status": (_c.c_int, [_P]),
     "fh_selftest_bounded_wait": (_c.c_int, [_c.c_uint32, _P]),
 }
@@ -242,6 +244,39 @@ def fh_gelu_bf16(x: torch.Tensor, y: torch.Tensor, stream=None) -> None:
     if x.numel() != y.numel() or not x.is_contiguous() or not y.is_contiguous():
         raise ValueError("x and y must be contiguous with the same number of elements")
     _check(_lib.fh_gelu_bf16(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+
+
+def fh_quantize_int8_rows(x: torch.Tensor, q: torch.Tensor, scales: torch.Tensor, stream=None) -> None:
+    """Per-row symmetric INT8: BF16 x [rows, d] (row stride x.stride(0)) -> q int8 [rows, d], scales FP32 [rows]."""
+    _need(x, _BF16, "x", 2)
+    _need(q, (torch.int8,), "q", 2)
+    _need(scales, (torch.float32,), "scales", 1)
+    rows, d = x.shape
+    if x.stride(1) != 1 or not q.is_contiguous() or not scales.is_contiguous():
+        raise ValueError("x needs unit column stride; q and scales must be contiguous")
+    if tuple(q.shape) != (rows, d) or scales.numel() != rows:
+        raise ValueError("shape mismatch: q [rows, d], scales [rows]")
+    _check(_lib.fh_quantize_int8_rows(_ptr(x), rows, d, x.stride(0), _ptr(q), _ptr(scales), _stream(stream)))
+
+
+def fh_int8_attention_scores(q: torch.Tensor, q_scales: torch.Tensor, k: torch.Tensor, k_scales: torch.Tensor,
+                             sm_scale: float, s: torch.Tensor, stream=None) -> None:
+    """S [heads, tq, tk] FP32 = (acc * (s_q * sm_scale)) * s_k for INT8 q [heads, tq, d], k [heads, tk, d]."""
+    _need(q, (torch.int8,), "q", 3)
+    _need(k, (torch.int8,), "k", 3)
+    _need(q_scales, (torch.float32,), "q_scales")
+    _need(k_scales, (torch.float32,), "k_scales")
+    _need(s, (torch.float32,), "s", 3)
+    for t, n in ((q, "q"), (k, "k"), (q_scales, "q_scales"), (k_scales, "k_scales"), (s, "s")):
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    heads, tq, d = q.shape
+    tk = k.shape[1]
+    if (k.shape[0] != heads or k.shape[2] != d or tuple(s.shape) != (heads, tq, tk)
+            or q_scales.numel() != heads * tq or k_scales.numel() != heads * tk):
+        raise ValueError("shape mismatch: q [H, tq, d], k [H, tk, d], scales [H, t], s [H, tq, tk]")
+    _check(_lib.fh_int8_attention_scores(_ptr(q), _ptr(q_scales), _ptr(k), _ptr(k_scales), float(sm_scale),
+                                         _ptr(s), heads, tq, tk, d, _stream(stream)))
 
 
 def fh_selftest_bounded_wait(limit_us: int, stream=None) -> None:

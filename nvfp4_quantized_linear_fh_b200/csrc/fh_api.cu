@@ -233,6 +233,53 @@ int fh_gelu_bf16(const uint16_t* x_dev, uint16_t* y_dev, int64_t n, fh_stream_t 
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_gelu_bf16 launch");
 }
 
+int fh_quantize_int8_rows(const uint16_t* x_dev, int64_t rows, int64_t d, int64_t ldx, int8_t* q_dev,
+                          float* scales_dev, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (rows < 0 || d <= 0 || d % 8 != 0 || ldx < d || ldx % 8 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_quantize_int8_rows: need rows >= 0, d > 0, d %% 8 == 0, ldx >= d, ldx %% 8 == 0%s");
+  if (rows == 0) return FH_OK;
+  if (x_dev == nullptr || q_dev == nullptr || scales_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_quantize_int8_rows: null pointer%s");
+  if (!aligned16(x_dev) || !aligned16(q_dev) || (reinterpret_cast<uintptr_t>(scales_dev) & 3u) != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_quantize_int8_rows: x and q must be 16-byte aligned, scales 4-byte aligned%s");
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_int8_quantize_rows(x_dev, rows, d, ldx, q_dev, scales_dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_quantize_int8_rows launch");
+}
+
+int fh_int8_attention_scores(const int8_t* q_dev, const float* q_scales_dev, const int8_t* k_dev,
+                             const float* k_scales_dev, float sm_scale, float* s_dev, int64_t heads, int64_t tq,
+                             int64_t tk, int64_t d, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!isfinite(sm_scale))
+    return fail(FH_ERR_INVALID_ARG, "fh_int8_attention_scores: sm_scale must be finite%s");
+  if (heads < 0 || tq < 0 || tk < 0 || d <= 0 || d % 16 != 0 || tk % 4 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_int8_attention_scores: need heads, tq, tk >= 0, d > 0, d %% 16 == 0, tk %% 4 == 0%s");
+  if (heads > 0x7FFFFFFF || tq > 0x7FFFFFFF || tk > 0x7FFFFFFF || d > 65536)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_int8_attention_scores: heads, tq, tk must fit in 31 bits and d <= 65536%s");
+  if (heads == 0 || tq == 0 || tk == 0) return FH_OK;
+  if (heads * ((tq + 127) / 128) * ((tk + 255) / 256) > 0x7FFFFFFF || tq * tk * 4 >= ((int64_t)1 << 40) ||
+      tq * d >= ((int64_t)1 << 40) || tk * d >= ((int64_t)1 << 40))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_int8_attention_scores: tensor too large%s");
+  if (q_dev == nullptr || q_scales_dev == nullptr || k_dev == nullptr || k_scales_dev == nullptr ||
+      s_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_int8_attention_scores: null pointer%s");
+  if (!aligned16(q_dev) || !aligned16(k_dev) || !aligned16(s_dev))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_int8_attention_scores: q, k and s must be 16-byte aligned%s");
+  if (int st = check_device()) return st;
+  const char* why = nullptr;
+  cudaError_t e = fh::launch_int8_scores(q_dev, q_scales_dev, k_dev, k_scales_dev, sm_scale, s_dev, heads, tq, tk,
+                                         d, (cudaStream_t)stream, &why);
+  if (e == cudaErrorNotSupported && why != nullptr)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_int8_attention_scores: %s", why);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_int8_attention_scores launch");
+}
+
 int fh_selftest_bounded_wait(uint32_t limit_us, fh_stream_t stream) {
   g_last_error[0] = 0;
   if (limit_us == 0 || limit_us > 2000000u)
@@ -245,11 +292,12 @@ int fh_selftest_bounded_wait(uint32_t limit_us, fh_stream_t stream) {
 int fh_device_status(fh_stream_t stream) {
   g_last_error[0] = 0;
   if (int st = check_device()) return st;
-  unsigned int bits = 0, qbits = 0;
+  unsigned int bits = 0, qbits = 0, ibits = 0;
   cudaError_t e = fh::read_and_clear_device_error(&bits, (cudaStream_t)stream);
   if (e == cudaSuccess) e = fh::read_and_clear_quant_error(&qbits);
+  if (e == cudaSuccess) e = fh::read_and_clear_int8_error(&ibits);
   if (e != cudaSuccess) return cuda_fail(e, "fh_device_status");
-  bits |= qbits;
+  bits |= qbits | ibits;
   if (bits & fh::kDevErrTimeout)
     return fail(FH_ERR_TIMEOUT, "a kernel gave up on a bounded on-chip wait%s");
   return FH_OK;

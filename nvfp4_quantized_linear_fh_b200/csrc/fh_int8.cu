@@ -1,0 +1,536 @@
+// fh_int8.cu -- INT8 query/key quantization and INT8 attention scores on the
+// sm_100a tensor cores.
+//
+// FastH3 Trim (comfyui-wiki news), "How fast it runs": the FP8 path of the
+// RTX 4090 quantizes the query and the key to INT8 to compute the attention
+// scores.  The pages fix neither the granularity nor the rounding; this file
+// takes one symmetric scale per row (one token of one head):
+//   s = fp32(amax_row / 127),  q = clamp(rne(fp32(x / s)), -127, 127)
+// (IEEE single divisions; s = q = 0 for an all-zero row), and the scores
+//   S[h, i, j] = ((float(acc) * (s_q[h, i] * sm_scale)) * s_k[h, j]),
+//   acc = sum_d q[h, i, d] * k[h, j, d]   (exact, INT32 on the tensor cores).
+//
+// Score kernel: persistent, warp-specialized, one CTA per SM, 192 threads.
+//   warp 0      TMA producer: per tile, the 128 query rows and 256 key rows
+//               (128-byte rows, 128-byte swizzle) of one head, one 128-element
+//               slice of d per stage; 3-D tensor maps (d, token, head) so that
+//               rows past a head's token count read as zero.
+//   warp 1      allocates TMEM (two 256-column INT32 accumulators) and issues
+//               tcgen05.mma kind::i8 (M = 128, N = 256, K = 32): four per stage.
+//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, the FP32 scaling,
+//               128-byte-swizzled staging and 3-D TMA stores (clipped at each
+//               head's bounds), while the MMA warp fills the other accumulator.
+// No TMA load uses cluster multicast.  Every mbarrier wait is bounded; on
+// expiry the kernel sets its error word and drains what it issued.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fh_internal.h"
+
+namespace fh {
+
+namespace {
+
+__device__ unsigned int g_int8_error = 0;
+
+// ---- row quantizer -------------------------------------------------------------
+
+// One warp per row; d % 8 == 0 (16-byte loads of 8 BF16 values).
+__global__ void __launch_bounds__(256) int8_quantize_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                                 int64_t d, int64_t ldx, int8_t* __restrict__ q,
+                                                                 float* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t r = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
+    const uint16_t* xr = x + r * ldx;
+    uint32_t mx = 0;  // max magnitude bits (BF16 magnitudes order like their bits)
+    for (int64_t c = 8 * lane; c < d; c += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(xr + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mx = max(mx, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    const float s = __fdiv_rn(__uint_as_float(mx << 16), 127.0f);
+    if (lane == 0) scales[r] = s;
+    int8_t* qr = q + r * d;
+    for (int64_t c = 8 * lane; c < d; c += 256) {
+      const uint4 v = *reinterpret_cast<const uint4*>(xr + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t out[2] = {0, 0};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const float xv = __uint_as_float(hlf ? (w[k] & 0xFFFF0000u) : (w[k] << 16));
+          int qi = 0;
+          if (s > 0.0f) qi = min(127, max(-127, __float2int_rn(__fdiv_rn(xv, s))));
+          out[k >> 1] |= ((uint32_t)qi & 0xFFu) << (8 * (2 * (k & 1) + hlf));
+        }
+      }
+      *reinterpret_cast<uint2*>(qr + c) = make_uint2(out[0], out[1]);
+    }
+  }
+}
+
+// ---- PTX helpers for the score kernel --------------------------------------------
+
+__device__ __forceinline__ uint32_t s_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait (~4 s, or until another role gave up): sets the error word and
+// the CTA's abort flag on expiry.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+  if (bar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 1; i < (1u << 30); ++i) {
+    if (bar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 0u) {
+      if (*abort) return false;
+      if (now_ns() - t0 > 4000000000ull) break;
+    }
+  }
+  atomicOr(&g_int8_error, (unsigned)kDevErrTimeout);
+  *abort = 1;
+  return false;
+}
+
+// Drain wait: bounded by time only (~1 s), ignores the abort flag.
+__device__ __forceinline__ void bar_drain(uint32_t bar, uint32_t parity) {
+  if (bar_try_wait(bar, parity)) return;
+  const uint64_t t0 = now_ns();
+  for (uint32_t i = 1; i < (1u << 30); ++i) {
+    if (bar_try_wait(bar, parity)) return;
+    if ((i & 255u) == 0u && now_ns() - t0 > 1000000000ull) break;
+  }
+  atomicOr(&g_int8_error, (unsigned)kDevErrTimeout);
+}
+
+__device__ __forceinline__ bool elect() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y, int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y), "r"(z)
+               : "memory");
+}
+
+// K-major operand descriptor, 128-byte rows in 1024-byte swizzle atoms.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  uint64_t dsc = (uint64_t)((addr >> 4) & 0x3FFFu);
+  dsc |= (uint64_t)1u << 16;
+  dsc |= (uint64_t)(1024u >> 4) << 32;
+  dsc |= (uint64_t)1u << 46;
+  dsc |= (uint64_t)2u << 61;
+  return dsc;
+}
+
+__device__ __forceinline__ void tmem_load_32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+        "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+        "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+        "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+// Completes the tcgen05.ld that wrote v; the registers are tied to the wait so
+// that no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_wait_32(uint32_t (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                 "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
+                 "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
+}
+
+// ---- score kernel ----------------------------------------------------------------
+
+constexpr int kTM = 128;                  // query rows per tile
+constexpr int kTN = 256;                  // key rows per tile
+constexpr int kSK = 128;                  // d elements (bytes) per stage
+constexpr int kMmaKI8 = 32;               // K of one tcgen05.mma kind::i8
+constexpr int kStagesI8 = 2;
+constexpr int kABytesI8 = kTM * kSK;      // 16384
+constexpr int kBBytesI8 = kTN * kSK;      // 32768
+constexpr int kEpiWarpsI8 = 8;                      // two per TMEM lane quadrant, one per column half
+constexpr int kThreadsI8 = 32 * (2 + kEpiWarpsI8);  // 320
+constexpr int kEpiCols = kTN / 2;                   // accumulator columns per epilogue warp
+constexpr int kOutBufs = 3;                         // staging buffers (stores in flight) per epilogue warp
+constexpr int kOutCols = 32;              // FP32 columns per TMA store box (128 bytes)
+constexpr int kOutBufBytes = 32 * kOutCols * 4;     // 4096
+constexpr int kOffAI8 = 0;
+constexpr int kOffBI8 = kOffAI8 + kStagesI8 * kABytesI8;
+constexpr int kOffOutI8 = kOffBI8 + kStagesI8 * kBBytesI8;
+constexpr int kOffKsI8 = kOffOutI8 + kEpiWarpsI8 * kOutBufs * kOutBufBytes;
+constexpr int kOffBarI8 = kOffKsI8 + kEpiWarpsI8 * kEpiCols * 4;
+constexpr int kNumBarsI8 = 2 * kStagesI8 + 4 + 1;  // full, empty; acc full (2), acc empty (2); drain
+constexpr int kSmemI8 = kOffBarI8 + kNumBarsI8 * 8 + 16 + 1024;
+// tcgen05.mma kind::i8: D S32 (bits 4-5 = 2), A and B signed 8-bit (1 at bits
+// 7 and 10), both K-major, N >> 3 at bit 17, M >> 4 at bit 24.
+constexpr uint32_t kIdescI8 = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kTN >> 3) << 17) |
+                              ((uint32_t)(kTM >> 4) << 24);
+static_assert(kSmemI8 <= 232448, "shared memory budget");
+static_assert(kOffBI8 % 1024 == 0 && kOffOutI8 % 1024 == 0, "alignment");
+
+struct ScoreParams {
+  const float* q_scales;
+  const float* k_scales;
+  float sm_scale;
+  int heads, tq, tk;
+  int m_tiles, n_tiles, num_tiles, k_stages;
+};
+
+struct RingI8 {
+  int slot = 0;
+  uint32_t phase = 0;
+  __device__ __forceinline__ void next(int n) {
+    if (++slot == n) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+};
+
+__global__ void __launch_bounds__(kThreadsI8, 1)
+    int8_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmS, const ScoreParams p) {
+  constexpr int S = kStagesI8;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = s_u32(smem);
+  const uint32_t bar0 = sbase + kOffBarI8;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBarI8 + kNumBarsI8 * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBarI8 + kNumBarsI8 * 8 + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      bar_init(full_bar(s), 1);
+      bar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      bar_init(accf_bar(a), 1);
+      bar_init(acce_bar(a), kEpiWarpsI8);
+    }
+    bar_init(drain_bar, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmS)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(s_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ===================== TMA producer =====================
+    RingI8 st;
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      const int h = t / (p.m_tiles * p.n_tiles), rem = t % (p.m_tiles * p.n_tiles);
+      const int m0 = (rem / p.n_tiles) * kTM, n0 = (rem % p.n_tiles) * kTN;
+      for (int kt = 0; kt < p.k_stages; ++kt) {
+        if (!__all_sync(0xFFFFFFFFu, bar_wait(empty_bar(st.slot), st.phase ^ 1u, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if (elect()) {
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full_bar(st.slot)),
+                       "r"((uint32_t)(kABytesI8 + kBBytesI8))
+                       : "memory");
+          tma_load_3d(sbase + kOffAI8 + st.slot * kABytesI8, &tmQ, full_bar(st.slot), kt * kSK, m0, h);
+          tma_load_3d(sbase + kOffBI8 + st.slot * kBBytesI8, &tmK, full_bar(st.slot), kt * kSK, n0, h);
+        }
+        __syncwarp();
+        st.next(S);
+      }
+    }
+    for (int s = 0; s < S; ++s) bar_drain(full_bar(s), (s < st.slot) ? st.phase : (st.phase ^ 1u));
+  } else if (warp == 1) {
+    // ===================== MMA issuer =====================
+    RingI8 st;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    bool ok = true;
+    const uint64_t adesc0 = sw128_desc(sbase + kOffAI8);
+    const uint64_t bdesc0 = sw128_desc(sbase + kOffBI8);
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      if (!__all_sync(0xFFFFFFFFu, bar_wait(acce_bar(acc), acc_phase ^ 1u, abort_flag))) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kTN);
+      for (int kt = 0; kt < p.k_stages; ++kt) {
+        if (!__all_sync(0xFFFFFFFFu, bar_wait(full_bar(st.slot), st.phase, abort_flag))) {
+          ok = false;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint64_t adesc = adesc0 + (uint64_t)((st.slot * kABytesI8) >> 4);
+        const uint64_t bdesc = bdesc0 + (uint64_t)((st.slot * kBBytesI8) >> 4);
+        if (elect()) {
+#pragma unroll
+          for (int k = 0; k < kSK / kMmaKI8; ++k)
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                "l"(adesc + (uint64_t)(k * kMmaKI8 / 16)), "l"(bdesc + (uint64_t)(k * kMmaKI8 / 16)),
+                "r"(kIdescI8), "r"((kt | k) != 0 ? 1u : 0u)
+                : "memory");
+          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           empty_bar(st.slot))
+                       : "memory");
+        }
+        __syncwarp();
+        st.next(S);
+      }
+      if (!ok) break;
+      if (elect())
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         accf_bar(acc))
+                     : "memory");
+      __syncwarp();
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (elect())
+      asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(drain_bar)
+                   : "memory");
+    __syncwarp();
+    bar_drain(drain_bar, 0);
+  } else {
+    // ===================== epilogue =====================
+    // Warp ew = warp - 2 reads TMEM lane quadrant warp % 4 (rows 32q .. 32q+31
+    // of the tile) and accumulator columns [half * 128, half * 128 + 128).
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int col0 = (ew >> 2) * kEpiCols;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    uint8_t* out_buf = smem + kOffOutI8 + ew * kOutBufs * kOutBufBytes;
+    float* ks_s = reinterpret_cast<float*>(smem + kOffKsI8) + ew * kEpiCols;
+    int acc = 0, buf = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+      const int h = t / (p.m_tiles * p.n_tiles), rem = t % (p.m_tiles * p.n_tiles);
+      const int m0 = (rem / p.n_tiles) * kTM, n0 = (rem % p.n_tiles) * kTN + col0;
+      const int row = m0 + 32 * q + lane;  // this thread's query row within the head
+      const bool rows_live = m0 + 32 * q < p.tq;
+      // This warp's copy of its columns' key scales (4 per lane).
+#pragma unroll
+      for (int i = lane; i < kEpiCols; i += 32)
+        ks_s[i] = (n0 + i < p.tk) ? p.k_scales[(size_t)h * p.tk + n0 + i] : 0.0f;
+      const float qs = (row < p.tq) ? p.q_scales[(size_t)h * p.tq + row] * p.sm_scale : 0.0f;
+      __syncwarp();
+      if (!__all_sync(0xFFFFFFFFu, bar_wait(accf_bar(acc), acc_phase, abort_flag))) break;
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const uint32_t tcol = tmem_base + lane_base + (uint32_t)(acc * kTN + col0);
+      // Chunk c's TMEM load is in flight while chunk c - 1 is scaled and stored.
+      uint32_t va[32], vb[32];
+      tmem_load_32(tcol, va);
+      tmem_wait_32(va);
+      auto emit = [&](const uint32_t(&v)[32], int c) {
+        float o[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = ((float)(int32_t)v[j] * qs) * ks_s[c * kOutCols + j];
+        // Reuse a staging buffer only after its previous store has read it.
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kOutBufs - 1) : "memory");
+        __syncwarp();
+        uint8_t* sb = out_buf + buf * kOutBufBytes;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t chunk = (uint32_t)i ^ ((uint32_t)lane & 7u);  // 128-byte swizzle
+          *reinterpret_cast<float4*>(sb + lane * 128 + chunk * 16) =
+              make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        // Boxes past the head's tokens or keys are not stored; partial boxes are
+        // clipped by the tensor map.
+        if (lane == 0 && rows_live && n0 + c * kOutCols < p.tk) {
+          tma_store_3d(&tmS, s_u32(sb), n0 + c * kOutCols, m0 + 32 * q, h);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        if (++buf == kOutBufs) buf = 0;
+      };
+      static_assert(kEpiCols / kOutCols == 4, "the pipelined epilogue below handles four chunks");
+      tmem_load_32(tcol + 32, vb);
+      emit(va, 0);
+      tmem_wait_32(vb);
+      tmem_load_32(tcol + 64, va);
+      emit(vb, 1);
+      tmem_wait_32(va);
+      tmem_load_32(tcol + 96, vb);
+      emit(va, 2);
+      tmem_wait_32(vb);
+      // Every TMEM read of this accumulator is complete: release it to the MMA.
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce_bar(acc)) : "memory");
+      emit(vb, 3);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512));
+  }
+}
+
+// ---- host ----------------------------------------------------------------------
+
+typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn encode3() {
+  static EncodeFn fn = nullptr;
+  if (fn == nullptr) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map of a [heads][rows][inner] array with a box of box_inner x box_rows x 1.
+bool map3(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows, uint64_t heads,
+          uint64_t elem_bytes, uint32_t box_inner, uint32_t box_rows) {
+  EncodeFn fn = encode3();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {inner, rows, heads};
+  const cuuint64_t strides[2] = {inner * elem_bytes, inner * rows * elem_bytes};
+  const cuuint32_t box[3] = {box_inner, box_rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_int8_quantize_rows(const uint16_t* x, int64_t rows, int64_t d, int64_t ldx, int8_t* q,
+                                      float* scales, cudaStream_t s) {
+  const int64_t blocks_needed = (rows + 7) / 8;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  const int grid = (int)(blocks_needed < cap ? (blocks_needed > 0 ? blocks_needed : 1) : cap);
+  int8_quantize_rows_kernel<<<grid, 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int8_t* k, const float* k_scales,
+                               float sm_scale, float* out, int64_t heads, int64_t tq, int64_t tk, int64_t d,
+                               cudaStream_t s, const char** why) {
+  CUtensorMap tmQ, tmK, tmS;
+  if (!map3(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)d, (uint64_t)tq, (uint64_t)heads, 1, kSK, kTM) ||
+      !map3(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, k, (uint64_t)d, (uint64_t)tk, (uint64_t)heads, 1, kSK, kTN) ||
+      !map3(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, (uint64_t)tk, (uint64_t)tq, (uint64_t)heads, 4, kOutCols,
+            32)) {
+    *why = "cuTensorMapEncodeTiled failed (driver entry point missing or a layout rule violated)";
+    return cudaErrorNotSupported;
+  }
+  ScoreParams p;
+  p.q_scales = q_scales;
+  p.k_scales = k_scales;
+  p.sm_scale = sm_scale;
+  p.heads = (int)heads;
+  p.tq = (int)tq;
+  p.tk = (int)tk;
+  p.m_tiles = (int)((tq + kTM - 1) / kTM);
+  p.n_tiles = (int)((tk + kTN - 1) / kTN);
+  p.num_tiles = (int)heads * p.m_tiles * p.n_tiles;
+  p.k_stages = (int)((d + kSK - 1) / kSK);  // the last stage's columns past d read as zero
+  static int configured = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured != dev) {
+    cudaError_t e = cudaFuncSetAttribute(int8_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemI8);
+    if (e != cudaSuccess) return e;
+    configured = dev;
+  }
+  const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
+  int8_scores_kernel<<<grid, kThreadsI8, kSmemI8, s>>>(tmQ, tmK, tmS, p);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_int8_error(unsigned int* bits) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_int8_error, sizeof v);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyToSymbol(g_int8_error, &zero, sizeof zero);
+  *bits = v;
+  return e;
+}
+
+}  // namespace fh

@@ -21,6 +21,9 @@ cudaError_t read_and_clear_device_error(unsigned int* bits, cudaStream_t s);
 // The quantizer's error word (fh_quant.cu); call after the stream is synchronized.
 cudaError_t read_and_clear_quant_error(unsigned int* bits);
 
+// The INT8 score kernel's error word (fh_int8.cu); call after the stream is synchronized.
+cudaError_t read_and_clear_int8_error(unsigned int* bits);
+
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
@@ -69,5 +72,17 @@ cudaError_t launch_nvfp4_linear_gelu_quant(const uint8_t* a_codes, const uint8_t
                                            const uint16_t* bias, float out_g, uint8_t* out_codes,
                                            uint8_t* out_scales, unsigned long long* out_clip, int64_t M,
                                            int64_t N, int64_t K, cudaStream_t s, const char** why);
+
+// INT8 query/key path (fh_int8.cu).  Arguments are validated by the caller.
+// Per-row symmetric INT8 quantization of BF16 rows (d % 8 == 0).
+cudaError_t launch_int8_quantize_rows(const uint16_t* x, int64_t rows, int64_t d, int64_t ldx, int8_t* q,
+                                      float* scales, cudaStream_t s);
+// S[h, i, j] = (float(q_i . k_j) * (s_q[i] * sm_scale)) * s_k[j] in FP32 for
+// q [heads, tq, d], k [heads, tk, d] INT8 and out [heads, tq, tk] FP32 (d % 16 == 0,
+// tk % 4 == 0).  cudaErrorNotSupported with a message in *why when the tensor
+// maps cannot be built.
+cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int8_t* k, const float* k_scales,
+                               float sm_scale, float* out, int64_t heads, int64_t tq, int64_t tk, int64_t d,
+                               cudaStream_t s, const char** why);
 
 }  // namespace fh

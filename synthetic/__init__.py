@@ -227,3 +227,20 @@ def random_bf16(seed_key, shape, std: float = 1.0) -> np.ndarray:
     """Plain N(0, std^2) BF16 bits of any shape (edge-case tests)."""
     n = int(np.prod(shape))
     return to_bf16_bits(normal(derive_seed(*seed_key), 0, n) * std).reshape(shape)
+
+
+def attention_qk(heads: int, tokens: int, d: int, which: str, seed: int = 0) -> np.ndarray:
+    """Query or key activations of shape [heads, tokens, d] as BF16 bits.
+
+    Each (head, channel) has its own spread, exp(N(0, 0.5^2)), and one channel
+    in 32 of every head is an outlier channel with 8x that spread; that is the
+    channel-wise outlier structure of attention queries and keys that
+    per-token INT8 scales must absorb.  Every tenth token is scaled by 4, so
+    rows differ in range as well."""
+    n = heads * tokens * d
+    z = normal(derive_seed("attn", which, seed, heads, tokens, d), 0, n).reshape(heads, tokens, d)
+    spread = np.exp(0.5 * normal(derive_seed("attn-spread", which, seed, heads, d), 0, heads * d)).reshape(heads, 1, d)
+    outlier = (u64(derive_seed("attn-outlier", which, seed, heads, d), 0, heads * d) % 32 == 0).reshape(heads, 1, d)
+    spread = spread * np.where(outlier, 8.0, 1.0)
+    row = np.where(np.arange(tokens) % 10 == 0, 4.0, 1.0).reshape(1, tokens, 1)
+    return to_bf16_bits(z * spread * row)

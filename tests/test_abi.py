@@ -106,6 +106,25 @@ def test_argument_validation_without_gpu(lib):
     assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, None, fake, None, 128, 256, 128, None) == 1  # null codes
     assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, P(24), fake, None, 128, 256, 128, None) == 2
     assert f(fake, fake, 1.0, fake, fake, 1.0, None, 1.0, fake, fake, None, 0, 256, 128, None) == 0   # empty
+    r = lib.fh_quantize_int8_rows
+    r.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P, P]
+    assert r(fake, 4, 12, 12, fake, fake, None) == 2       # d % 8
+    assert r(fake, 4, 16, 8, fake, fake, None) == 2        # ldx < d
+    assert r(fake, 4, 16, 20, fake, fake, None) == 2       # ldx % 8
+    assert r(None, 4, 16, 16, fake, fake, None) == 1       # null x
+    assert r(fake, 4, 16, 16, P(24), fake, None) == 2      # q misaligned
+    assert r(fake, 4, 16, 16, fake, P(18), None) == 2      # scales misaligned
+    assert r(fake, 0, 16, 16, fake, fake, None) == 0       # empty
+    s = lib.fh_int8_attention_scores
+    s.argtypes = [P, P, P, P, ctypes.c_float, P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P]
+    assert s(fake, fake, fake, fake, 1.0, fake, 2, 100, 256, 120, None) == 2   # d % 16
+    assert s(fake, fake, fake, fake, 1.0, fake, 2, 100, 254, 128, None) == 2   # tk % 4
+    assert s(fake, fake, fake, fake, 1.0, fake, 2, 100, 256, 131072, None) == 2  # d too large for INT32 sums
+    assert s(fake, fake, fake, fake, float("nan"), fake, 2, 100, 256, 128, None) == 1
+    assert s(fake, None, fake, fake, 1.0, fake, 2, 100, 256, 128, None) == 1  # null q scales
+    assert s(fake, fake, P(40), fake, 1.0, fake, 2, 100, 256, 128, None) == 2  # k misaligned
+    assert s(fake, fake, fake, fake, 1.0, fake, 2, 0, 256, 128, None) == 0     # empty
+    assert s(fake, fake, fake, fake, 1.0, fake, 0, 100, 256, 128, None) == 0
     a = lib.fh_amax
     a.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P]
     assert a(fake, 3, 5, 4, fake, None) == 2
