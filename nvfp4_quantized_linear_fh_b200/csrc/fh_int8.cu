@@ -37,7 +37,14 @@ __device__ unsigned int g_int8_error = 0;
 
 // ---- row quantizer -------------------------------------------------------------
 
-// One warp per row; d % 8 == 0 (16-byte loads of 8 BF16 values).
+// The element decision shared by both row kernels: q = clamp(rne(x / s)).
+__device__ __forceinline__ uint32_t int8_code(float xv, float s) {
+  int qi = 0;
+  if (s > 0.0f) qi = min(127, max(-127, __float2int_rn(__fdiv_rn(xv, s))));
+  return (uint32_t)qi & 0xFFu;
+}
+
+// General form (any d % 8 == 0): one warp per row, two passes over the row.
 __global__ void __launch_bounds__(256) int8_quantize_rows_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                                  int64_t d, int64_t ldx, int8_t* __restrict__ q,
                                                                  float* __restrict__ scales) {
@@ -66,12 +73,74 @@ __global__ void __launch_bounds__(256) int8_quantize_rows_kernel(const uint16_t*
 #pragma unroll
         for (int hlf = 0; hlf < 2; ++hlf) {
           const float xv = __uint_as_float(hlf ? (w[k] & 0xFFFF0000u) : (w[k] << 16));
-          int qi = 0;
-          if (s > 0.0f) qi = min(127, max(-127, __float2int_rn(__fdiv_rn(xv, s))));
-          out[k >> 1] |= ((uint32_t)qi & 0xFFu) << (8 * (2 * (k & 1) + hlf));
+          out[k >> 1] |= int8_code(xv, s) << (8 * (2 * (k & 1) + hlf));
         }
       }
       *reinterpret_cast<uint2*>(qr + c) = make_uint2(out[0], out[1]);
+    }
+  }
+}
+
+// Register-resident form for d <= 2048: a group of G lanes holds RB rows of NC
+// 16-byte chunks per lane, so each row is read from HBM once and the loads of
+// RB rows are in flight together.  Chunks past d read as zero (they change no
+// maximum) and are not stored.
+template <int G, int NC, int RB>
+__global__ void __launch_bounds__(256) int8_rows_reg_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t d,
+                                                            int64_t ldx, int8_t* __restrict__ q,
+                                                            float* __restrict__ scales) {
+  static_assert(32 % G == 0 && NC >= 1 && RB >= 1, "group shape");
+  const int lane = threadIdx.x & 31, sub = lane % G;
+  constexpr int kGroupsPerBlock = 8 * (32 / G);
+  const int64_t gid = (int64_t)blockIdx.x * kGroupsPerBlock + (threadIdx.x >> 5) * (32 / G) + lane / G;
+  const int64_t stride = (int64_t)gridDim.x * kGroupsPerBlock * RB;
+  // The loop runs on the warp's first group (rw), so that all 32 lanes take the
+  // full-warp shuffles together; a group past the last row loads zeros and
+  // stores nothing.
+  for (int64_t r0 = gid * RB, rw = (gid - lane / G) * RB; rw < rows; r0 += stride, rw += stride) {
+    uint4 v[RB][NC];
+    uint32_t mx[RB];
+#pragma unroll
+    for (int b = 0; b < RB; ++b) {
+#pragma unroll
+      for (int i = 0; i < NC; ++i) {
+        const int64_t c = (int64_t)(sub + G * i) * 8;
+        v[b][i] = (r0 + b < rows && c < d) ? *reinterpret_cast<const uint4*>(x + (r0 + b) * ldx + c)
+                                           : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < RB; ++b) {
+      uint32_t m = 0;  // max magnitude bits (BF16 magnitudes order like their bits)
+#pragma unroll
+      for (int i = 0; i < NC; ++i) {
+        const uint32_t w[4] = {v[b][i].x, v[b][i].y, v[b][i].z, v[b][i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m = max(m, max(w[k] & 0x7FFFu, (w[k] >> 16) & 0x7FFFu));
+      }
+#pragma unroll
+      for (int o = G / 2; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+      mx[b] = m;
+    }
+#pragma unroll
+    for (int b = 0; b < RB; ++b) {
+      const int64_t r = r0 + b;
+      if (r >= rows) break;
+      const float sc = __fdiv_rn(__uint_as_float(mx[b] << 16), 127.0f);
+      if (sub == 0) scales[r] = sc;
+#pragma unroll
+      for (int i = 0; i < NC; ++i) {
+        const int64_t c = (int64_t)(sub + G * i) * 8;
+        if (c >= d) break;
+        const uint32_t w[4] = {v[b][i].x, v[b][i].y, v[b][i].z, v[b][i].w};
+        uint32_t out[2] = {0, 0};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          out[k >> 1] |= int8_code(__uint_as_float(w[k] << 16), sc) << (16 * (k & 1));
+          out[k >> 1] |= int8_code(__uint_as_float(w[k] & 0xFFFF0000u), sc) << (16 * (k & 1) + 8);
+        }
+        *reinterpret_cast<uint2*>(q + r * d + c) = make_uint2(out[0], out[1]);
+      }
     }
   }
 }
@@ -482,10 +551,30 @@ bool map3(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inn
 
 cudaError_t launch_int8_quantize_rows(const uint16_t* x, int64_t rows, int64_t d, int64_t ldx, int8_t* q,
                                       float* scales, cudaStream_t s) {
-  const int64_t blocks_needed = (rows + 7) / 8;
+  // Rows per block of each form; the grid covers the rows once, up to 8 blocks
+  // of 256 threads per SM, with a grid-stride loop beyond that.
   const int64_t cap = (int64_t)sm_count() * 8;
-  const int grid = (int)(blocks_needed < cap ? (blocks_needed > 0 ? blocks_needed : 1) : cap);
-  int8_quantize_rows_kernel<<<grid, 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  auto grid_for = [&](int64_t rows_per_block) {
+    const int64_t need = (rows + rows_per_block - 1) / rows_per_block;
+    return (int)(need < cap ? (need > 0 ? need : 1) : cap);
+  };
+  const int64_t chunks = d / 8;  // 16-byte chunks per row
+  if (chunks <= 4)
+    int8_rows_reg_kernel<4, 1, 2><<<grid_for(8 * 8 * 2), 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  else if (chunks <= 8)
+    int8_rows_reg_kernel<8, 1, 2><<<grid_for(8 * 4 * 2), 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  else if (chunks <= 16)
+    int8_rows_reg_kernel<16, 1, 2><<<grid_for(8 * 2 * 2), 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  else if (chunks <= 32)
+    int8_rows_reg_kernel<32, 1, 2><<<grid_for(8 * 2), 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  else if (chunks <= 64)
+    int8_rows_reg_kernel<32, 2, 2><<<grid_for(8 * 2), 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  else if (chunks <= 128)
+    int8_rows_reg_kernel<32, 4, 1><<<grid_for(8), 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  else if (chunks <= 256)
+    int8_rows_reg_kernel<32, 8, 1><<<grid_for(8), 256, 0, s>>>(x, rows, d, ldx, q, scales);
+  else
+    int8_quantize_rows_kernel<<<grid_for(8), 256, 0, s>>>(x, rows, d, ldx, q, scales);
   return cudaGetLastError();
 }
 

@@ -36,8 +36,13 @@ def _assert_rows_exact(x_bits, ldx=None):
     assert bad.size == 0, f"{len(bad)} INT8 codes differ, first at {bad[:5].tolist()}"
 
 
-@pytest.mark.parametrize("rows,d,ldx", [(1, 8, None), (300, 128, None), (257, 136, None),
-                                        (1000, 64, 72), (33, 2688, None)])
+# One case per launch form of the row quantizer (lanes per row x chunks per
+# lane: 4x1, 8x1, 16x1, 32x1, 32x2, 32x4, 32x8, and the general two-pass form),
+# ragged row counts, a row stride wider than d, and a size that needs the
+# grid-stride loop.
+@pytest.mark.parametrize("rows,d,ldx", [(1, 8, None), (77, 40, 48), (1000, 64, 72), (300, 128, None),
+                                        (257, 136, None), (3, 200, None), (20, 384, None), (130, 520, 528),
+                                        (9, 1024, None), (17, 2048, None), (33, 2688, None), (200000, 32, None)])
 def test_quantize_rows_bit_exact(rows, d, ldx):
     x = S.attention_qk(1, rows, d, "rows", seed=rows + d).reshape(rows, d)
     _assert_rows_exact(x, ldx)
