@@ -383,6 +383,144 @@ def bench_ffn(args):
         "outputs_bit_identical": identical}))
 
 
+ATTN = {"heads": 21, "tokens": 4096, "d": 128}
+
+
+def attn_score_bytes(H, tq, tk, d):
+    """Algorithmic bytes of one score launch: INT8 Q and K, their FP32 scales, FP32 scores."""
+    return H * (tq + tk) * (d + 4) + 4 * H * tq * tk
+
+
+def attn_quant_bytes(rows, d):
+    """Algorithmic bytes of one INT8 row-quantizer launch: BF16 in, INT8 codes and FP32 scales out."""
+    return rows * (3 * d + 4)
+
+
+def bench_attn(args):
+    """INT8 attention scores of the 2688-wide transformer's self-attention
+    (21 heads x d 128, 4096 queries x 4096 keys per head): per-row INT8
+    quantization of Q and of K, then the tensor-core score kernel writing FP32
+    S[h, i, j].  One step = quantize Q, quantize K, scores."""
+    import torch
+    import synthetic as S
+    import nvfp4_quantized_linear_fh_b200 as fh
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    H, T, d = ATTN["heads"], ATTN["tokens"], ATTN["d"]
+
+    def to_dev(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    qb, kb = S.attention_qk(H, T, d, "q", 1), S.attention_qk(H, T, d, "k", 1)
+    xq, xk = to_dev(qb.reshape(H * T, d)), to_dev(kb.reshape(H * T, d))
+    q8 = torch.empty((H, T, d), dtype=torch.int8, device=dev)
+    k8 = torch.empty_like(q8)
+    qs = torch.empty((H, T), dtype=torch.float32, device=dev)
+    ks = torch.empty_like(qs)
+    sc = torch.empty((H, T, T), dtype=torch.float32, device=dev)
+    sm_scale = float(np.float32(1.0 / np.sqrt(d)))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        fh.fh_quantize_int8_rows(xq, q8.view(H * T, d), qs.view(-1))
+        fh.fh_quantize_int8_rows(xk, k8.view(H * T, d), ks.view(-1))
+        fh.fh_int8_attention_scores(q8, qs, k8, ks, sm_scale, sc)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 200))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    sampler = ClockSampler(f"GPU-{torch.cuda.get_device_properties(dev).uuid}")
+    with sampler:
+        sampler.wait_first_sample()
+        sampler.mark_start()
+        for i in range(steps):
+            ev[i][0].record(stream)
+            fh.fh_quantize_int8_rows(xq, q8.view(H * T, d), qs.view(-1))
+            fh.fh_quantize_int8_rows(xk, k8.view(H * T, d), ks.view(-1))
+            ev[i][1].record(stream)
+            fh.fh_int8_attention_scores(q8, qs, k8, ks, sm_scale, sc)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        sampler.mark_end()
+    fh.fh_device_status()
+    t_quant = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)) * 1e-3 / steps
+    t_scores = sum(ev[i][1].elapsed_time(ev[i][2]) for i in range(steps)) * 1e-3 / steps
+    t_step = t_quant + t_scores
+    ops = 2.0 * H * T * T * d
+
+    # End to end: BF16 Q and K from pinned host memory, FP32 scores back to pinned host memory.
+    t_e2e, e_steps = float("nan"), 0
+    if not args.no_e2e:
+        xq_h = torch.empty_like(xq, device="cpu").pin_memory()
+        xk_h = torch.empty_like(xk, device="cpu").pin_memory()
+        xq_h.copy_(xq.cpu())
+        xk_h.copy_(xk.cpu())
+        s_h = torch.empty((H, T, T), dtype=torch.float32).pin_memory()
+        e_steps = 3
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(e_steps):
+            xq.copy_(xq_h, non_blocking=True)
+            xk.copy_(xk_h, non_blocking=True)
+            step()
+            s_h.copy_(sc, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = e0.elapsed_time(e1) * 1e-3 / e_steps
+
+    pk = peaks()
+    by = attn_score_bytes(H, T, T, d)
+    achieved = by / t_scores / 1e9
+    line = {
+        "metric": "INT8 attention scores: whole-step TOPS (quantize Q, quantize K, Q.K^T scaled to FP32)",
+        "value": ops / t_step / 1e12, "unit": "TOPS", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "s8 (INT32 accumulate, FP32 scores)", "data": "synthetic (seeded Q/K with outlier channels)",
+        "config": {"workload": f"attention scores {H} heads x {T} queries x {T} keys x d {d}", "heads": H,
+                   "tq": T, "tk": T, "d": d,
+                   "l2": "not flushed: each step writes 1.41 GB of scores (> L2)"},
+        "kernels_us": {"int8_quantize_rows (Q and K)": t_quant * 1e6, "int8_scores_kernel": t_scores * 1e6},
+        "roofline": {"bound": "hbm", "kernel": "int8_scores_kernel", "achieved": achieved, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "peak_source": pk["source"],
+                     "traffic": ATTN_TRAFFIC["bytes"] if attn_traffic_valid() else None,
+                     "algorithmic_bytes": by},
+        "quantizer": {"achieved_gbs": 2 * attn_quant_bytes(H * T, d) / t_quant / 1e9},
+        "e2e": {"value": ops / t_e2e / 1e12 if e_steps else None, "unit": "TOPS",
+                "h2d_bytes_per_step": 2 * H * T * d * 2, "d2h_bytes_per_step": 4 * H * T * T},
+        "gpu_launches": 3 * steps, "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        rows = T  # one whole head: a few seconds of oracle work
+        t0 = time.perf_counter()
+        oq, oqs = oracle.quantize_int8_rows(qb[0, :rows])
+        ok, oks = oracle.quantize_int8_rows(kb[0])
+        oracle.int8_scores(oq[None], oqs[None], ok[None], oks[None], sm_scale)
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": 2.0 * rows * T * d / dt / 1e12, "unit": "TOPS",
+                                "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+                                "sample": f"head 0 of {H}: its {rows} query and {T} key rows quantized, "
+                                          f"their {rows}x{T} scores"}
+    print(json.dumps(line))
+
+
+# DRAM bytes (read + write) of one int8_scores_kernel launch on the workload
+# above, from an ncu capture; valid only for the kernel source it was taken on.
+ATTN_TRAFFIC = {"bytes": 1375100160, "source_sha256": "0630d6dd00149ba6"}
+
+
+def attn_traffic_valid():
+    import hashlib
+    path = os.path.join(ROOT, "nvfp4_quantized_linear_fh_b200", "csrc", "fh_int8.cu")
+    with open(path, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()[:16]
+    return ATTN_TRAFFIC["bytes"] is not None and digest == ATTN_TRAFFIC["source_sha256"]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -395,14 +533,18 @@ def main():
     ap.add_argument("--M", type=int, default=WORKLOAD["M"],
                     help="token rows per GPU (profiling cases use fewer than the workload's 32768)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
-    ap.add_argument("--workload", default="qkv", choices=["qkv", "ffn"],
-                    help="qkv: the headline line (fused QKV layer); ffn: the FFN block, fused vs unfused epilogue")
+    ap.add_argument("--workload", default="qkv", choices=["qkv", "ffn", "attn"],
+                    help="qkv: the headline line (fused QKV layer); ffn: the FFN block, fused vs unfused "
+                         "epilogue; attn: INT8 query/key quantization and attention scores")
     ap.add_argument("--quick", action="store_true",
                     help="calibrate on the input batches only (setup shortcut for profiling cases)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.workload == "ffn":
         bench_ffn(args)
+        return
+    if args.workload == "attn":
+        bench_attn(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

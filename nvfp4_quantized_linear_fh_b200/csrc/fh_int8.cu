@@ -10,16 +10,19 @@
 //   S[h, i, j] = ((float(acc) * (s_q[h, i] * sm_scale)) * s_k[h, j]),
 //   acc = sum_d q[h, i, d] * k[h, j, d]   (exact, INT32 on the tensor cores).
 //
-// Score kernel: persistent, warp-specialized, one CTA per SM, 192 threads.
+// Score kernel: persistent, warp-specialized, one CTA per SM, 320 threads.
 //   warp 0      TMA producer: per tile, the 128 query rows and 256 key rows
 //               (128-byte rows, 128-byte swizzle) of one head, one 128-element
 //               slice of d per stage; 3-D tensor maps (d, token, head) so that
-//               rows past a head's token count read as zero.
+//               rows past a head's token count, and columns past d, read as zero.
 //   warp 1      allocates TMEM (two 256-column INT32 accumulators) and issues
 //               tcgen05.mma kind::i8 (M = 128, N = 256, K = 32): four per stage.
-//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, the FP32 scaling,
-//               128-byte-swizzled staging and 3-D TMA stores (clipped at each
-//               head's bounds), while the MMA warp fills the other accumulator.
+//   warps 2..9  epilogue, two warps per TMEM lane quadrant (one per half of the
+//               columns): pipelined tcgen05.ld, the FP32 scaling, a transpose
+//               through shared memory and coalesced 16-byte stores (four whole
+//               128-byte rows of S per instruction), while the MMA warp fills
+//               the other accumulator.  S is write-bound: coalesced stores from
+//               eight warps keep more of it in flight than per-SM TMA stores.
 // No TMA load uses cluster multicast.  Every mbarrier wait is bounded; on
 // expiry the kernel sets its error word and drains what it issued.
 #include <cuda.h>
@@ -217,13 +220,6 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y, int z) {
-  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(src), "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-
 // K-major operand descriptor, 128-byte rows in 1024-byte swizzle atoms.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
   uint64_t dsc = (uint64_t)((addr >> 4) & 0x3FFFu);
@@ -272,13 +268,12 @@ constexpr int kBBytesI8 = kTN * kSK;      // 32768
 constexpr int kEpiWarpsI8 = 8;                      // two per TMEM lane quadrant, one per column half
 constexpr int kThreadsI8 = 32 * (2 + kEpiWarpsI8);  // 320
 constexpr int kEpiCols = kTN / 2;                   // accumulator columns per epilogue warp
-constexpr int kOutBufs = 3;                         // staging buffers (stores in flight) per epilogue warp
-constexpr int kOutCols = 32;              // FP32 columns per TMA store box (128 bytes)
+constexpr int kOutCols = 32;              // FP32 columns per epilogue chunk (128 bytes)
 constexpr int kOutBufBytes = 32 * kOutCols * 4;     // 4096
 constexpr int kOffAI8 = 0;
 constexpr int kOffBI8 = kOffAI8 + kStagesI8 * kABytesI8;
 constexpr int kOffOutI8 = kOffBI8 + kStagesI8 * kBBytesI8;
-constexpr int kOffKsI8 = kOffOutI8 + kEpiWarpsI8 * kOutBufs * kOutBufBytes;
+constexpr int kOffKsI8 = kOffOutI8 + kEpiWarpsI8 * kOutBufBytes;
 constexpr int kOffBarI8 = kOffKsI8 + kEpiWarpsI8 * kEpiCols * 4;
 constexpr int kNumBarsI8 = 2 * kStagesI8 + 4 + 1;  // full, empty; acc full (2), acc empty (2); drain
 constexpr int kSmemI8 = kOffBarI8 + kNumBarsI8 * 8 + 16 + 1024;
@@ -292,6 +287,7 @@ static_assert(kOffBI8 % 1024 == 0 && kOffOutI8 % 1024 == 0, "alignment");
 struct ScoreParams {
   const float* q_scales;
   const float* k_scales;
+  float* out;
   float sm_scale;
   int heads, tq, tk;
   int m_tiles, n_tiles, num_tiles, k_stages;
@@ -310,7 +306,7 @@ struct RingI8 {
 
 __global__ void __launch_bounds__(kThreadsI8, 1)
     int8_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmS, const ScoreParams p) {
+                       const ScoreParams p) {
   constexpr int S = kStagesI8;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -339,7 +335,6 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmQ)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmK)) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmS)) : "memory");
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(s_u32(tmem_slot)),
@@ -436,21 +431,35 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
     const int q = warp & 3;
     const int col0 = (ew >> 2) * kEpiCols;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    uint8_t* out_buf = smem + kOffOutI8 + ew * kOutBufs * kOutBufBytes;
+    uint8_t* out_buf = smem + kOffOutI8 + ew * kOutBufBytes;
     float* ks_s = reinterpret_cast<float*>(smem + kOffKsI8) + ew * kEpiCols;
-    int acc = 0, buf = 0;
+    int acc = 0;
     uint32_t acc_phase = 0;
+    // The scales of a tile are loaded into registers one tile ahead, so that
+    // their global-load latency overlaps the previous tile's epilogue.
+    constexpr int kKsPerLane = kEpiCols / 32;
+    float ks_next[kKsPerLane], qs_next = 0.0f;
+    auto load_scales = [&](int t) {
+      const int h = t / (p.m_tiles * p.n_tiles), rem = t % (p.m_tiles * p.n_tiles);
+      const int m0 = (rem / p.n_tiles) * kTM, n0 = (rem % p.n_tiles) * kTN + col0;
+      const int row = m0 + 32 * q + lane;
+#pragma unroll
+      for (int i = 0; i < kKsPerLane; ++i) {
+        const int col = n0 + lane + 32 * i;
+        ks_next[i] = (col < p.tk) ? p.k_scales[(size_t)h * p.tk + col] : 0.0f;
+      }
+      qs_next = (row < p.tq) ? p.q_scales[(size_t)h * p.tq + row] : 0.0f;
+    };
+    if (blockIdx.x < p.num_tiles) load_scales(blockIdx.x);
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       const int h = t / (p.m_tiles * p.n_tiles), rem = t % (p.m_tiles * p.n_tiles);
       const int m0 = (rem / p.n_tiles) * kTM, n0 = (rem % p.n_tiles) * kTN + col0;
-      const int row = m0 + 32 * q + lane;  // this thread's query row within the head
-      const bool rows_live = m0 + 32 * q < p.tq;
       // This warp's copy of its columns' key scales (4 per lane).
 #pragma unroll
-      for (int i = lane; i < kEpiCols; i += 32)
-        ks_s[i] = (n0 + i < p.tk) ? p.k_scales[(size_t)h * p.tk + n0 + i] : 0.0f;
-      const float qs = (row < p.tq) ? p.q_scales[(size_t)h * p.tq + row] * p.sm_scale : 0.0f;
+      for (int i = 0; i < kKsPerLane; ++i) ks_s[lane + 32 * i] = ks_next[i];
+      const float qs = qs_next * p.sm_scale;
       __syncwarp();
+      if (t + (int)gridDim.x < p.num_tiles) load_scales(t + gridDim.x);
       if (!__all_sync(0xFFFFFFFFu, bar_wait(accf_bar(acc), acc_phase, abort_flag))) break;
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const uint32_t tcol = tmem_base + lane_base + (uint32_t)(acc * kTN + col0);
@@ -462,25 +471,28 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
         float o[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) o[j] = ((float)(int32_t)v[j] * qs) * ks_s[c * kOutCols + j];
-        // Reuse a staging buffer only after its previous store has read it.
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kOutBufs - 1) : "memory");
-        __syncwarp();
-        uint8_t* sb = out_buf + buf * kOutBufBytes;
+        // Transpose through a 128-byte-swizzled staging buffer (thread = row on
+        // the way in, eight lanes per row on the way out), so that every store
+        // instruction writes four whole 128-byte rows of S.
+        uint8_t* sb = out_buf;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const uint32_t chunk = (uint32_t)i ^ ((uint32_t)lane & 7u);  // 128-byte swizzle
+          const uint32_t chunk = (uint32_t)i ^ ((uint32_t)lane & 7u);
           *reinterpret_cast<float4*>(sb + lane * 128 + chunk * 16) =
               make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
-        // Boxes past the head's tokens or keys are not stored; partial boxes are
-        // clipped by the tensor map.
-        if (lane == 0 && rows_live && n0 + c * kOutCols < p.tk) {
-          tma_store_3d(&tmS, s_u32(sb), n0 + c * kOutCols, m0 + 32 * q, h);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        const int gcol = n0 + c * kOutCols + 4 * (lane & 7);  // tk % 4 == 0: a float4 never straddles tk
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          const float4 val =
+              *reinterpret_cast<const float4*>(sb + r * 128 + (((uint32_t)(lane & 7) ^ (uint32_t)(r & 7)) * 16));
+          const int grow = m0 + 32 * q + r;
+          if (grow < p.tq && gcol < p.tk)
+            *reinterpret_cast<float4*>(p.out + ((size_t)h * p.tq + grow) * p.tk + gcol) = val;
         }
-        if (++buf == kOutBufs) buf = 0;
+        __syncwarp();  // the buffer is rewritten by the next chunk
       };
       static_assert(kEpiCols / kOutCols == 4, "the pipelined epilogue below handles four chunks");
       tmem_load_32(tcol + 32, vb);
@@ -502,8 +514,6 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
         acc_phase ^= 1u;
       }
     }
-    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-    __syncwarp();
   }
 
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -581,17 +591,16 @@ cudaError_t launch_int8_quantize_rows(const uint16_t* x, int64_t rows, int64_t d
 cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int8_t* k, const float* k_scales,
                                float sm_scale, float* out, int64_t heads, int64_t tq, int64_t tk, int64_t d,
                                cudaStream_t s, const char** why) {
-  CUtensorMap tmQ, tmK, tmS;
+  CUtensorMap tmQ, tmK;
   if (!map3(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, (uint64_t)d, (uint64_t)tq, (uint64_t)heads, 1, kSK, kTM) ||
-      !map3(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, k, (uint64_t)d, (uint64_t)tk, (uint64_t)heads, 1, kSK, kTN) ||
-      !map3(&tmS, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, out, (uint64_t)tk, (uint64_t)tq, (uint64_t)heads, 4, kOutCols,
-            32)) {
+      !map3(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, k, (uint64_t)d, (uint64_t)tk, (uint64_t)heads, 1, kSK, kTN)) {
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or a layout rule violated)";
     return cudaErrorNotSupported;
   }
   ScoreParams p;
   p.q_scales = q_scales;
   p.k_scales = k_scales;
+  p.out = out;
   p.sm_scale = sm_scale;
   p.heads = (int)heads;
   p.tq = (int)tq;
@@ -609,7 +618,7 @@ cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int
     configured = dev;
   }
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
-  int8_scores_kernel<<<grid, kThreadsI8, kSmemI8, s>>>(tmQ, tmK, tmS, p);
+  int8_scores_kernel<<<grid, kThreadsI8, kSmemI8, s>>>(tmQ, tmK, p);
   return cudaGetLastError();
 }
 
