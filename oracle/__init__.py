@@ -1,4 +1,5 @@
-"""CPU oracle of the NVFP4 quantized linear layer (binding to fh_oracle.c).
+"""CPU oracle of the NVFP4 quantized linear layer (binding to fh_oracle.c), and
+numpy definitions of the INT8 query/key scores and of the AdaLN basis projection.
 
 TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline / reference legs may import this package.  It shares
@@ -230,3 +231,49 @@ def int8_scores(q8: np.ndarray, q_scales: np.ndarray, k8: np.ndarray, k_scales: 
 def int8_scores_tolerance(s_ref: np.ndarray) -> np.ndarray:
     """Three FP32 roundings of an exact product: 2e-6 relative (2^-21 = 4.8e-7 each), plus 1e-30."""
     return 2e-6 * np.abs(s_ref) + 1e-30
+
+
+# ---- AdaLN timestep conditioning through a shared low-rank basis -------------------
+# FastH3 Trim (comfyui-wiki news), "What Trim changes": AdaLN maps the 2,688-wide
+# time embedding to six modulation vectors per block; Trim replaces the per-block
+# projections with one shared 2,688 -> 16 basis followed by a small projection per
+# block, both stored in FP16.  Reading: the two maps are linear,
+#   code[b, j]       = sum_k basis[j, k] * e[b, k]                  (r = 16 values)
+#   mod[l, b, i]     = sum_j proj[l, i, j] * code[b, j] + bias[l, i] (6 * 2688 values)
+# with BF16 embeddings, FP16 weights and exact (binary64) arithmetic here.
+
+def f16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """IEEE half bits -> float64 (exact)."""
+    return np.asarray(bits, dtype=np.uint16).view(np.float16).astype(np.float64)
+
+
+def adaln_code(e_bits: np.ndarray, basis_bits: np.ndarray) -> np.ndarray:
+    """code [bt, r] = e [bt, d] (BF16 bits) times basis^T, basis [r, d] (FP16 bits), in binary64."""
+    e = (np.asarray(e_bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+    return e @ f16_to_f64(basis_bits).T
+
+
+def adaln_modulation(code: np.ndarray, proj_bits: np.ndarray, bias_bits) -> np.ndarray:
+    """mod [L, bt, n] = proj [L, n, r] (FP16 bits) applied to code [bt, r], plus bias [L, n] (FP16 bits)."""
+    proj = f16_to_f64(proj_bits)
+    out = np.einsum("lir,br->lbi", proj, code)
+    if bias_bits is not None:
+        out = out + f16_to_f64(bias_bits)[:, None, :]
+    return out
+
+
+def adaln_tolerance(e_bits, basis_bits, proj_bits, bias_bits) -> np.ndarray:
+    """Worst-case bound for FP32 evaluation of the two maps in any summation order
+    (Higham's dot-product bound, gamma_n = n u / (1 - n u), u = 2^-24, applied to the
+    code and then to the projection):  |err| <= (gamma_d + gamma_{r+1} + gamma_d
+    gamma_{r+1}) * M, where M is the same expression evaluated on absolute values."""
+    e = np.abs((np.asarray(e_bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64))
+    code_abs = e @ np.abs(f16_to_f64(basis_bits)).T
+    m = np.einsum("lir,br->lbi", np.abs(f16_to_f64(proj_bits)), code_abs)
+    if bias_bits is not None:
+        m = m + np.abs(f16_to_f64(bias_bits))[:, None, :]
+    u = 2.0 ** -24
+    d, r = np.shape(e_bits)[1], np.shape(basis_bits)[0]
+    g1 = d * u / (1 - d * u)
+    g2 = (r + 1) * u / (1 - (r + 1) * u)
+    return (g1 + g2 + g1 * g2) * m * (1 + 1e-12) + 1e-37

@@ -244,3 +244,25 @@ def attention_qk(heads: int, tokens: int, d: int, which: str, seed: int = 0) -> 
     spread = spread * np.where(outlier, 8.0, 1.0)
     row = np.where(np.arange(tokens) % 10 == 0, 4.0, 1.0).reshape(1, tokens, 1)
     return to_bf16_bits(z * spread * row)
+
+
+def to_f16_bits(x: np.ndarray) -> np.ndarray:
+    """float64 -> IEEE half bits (numpy's conversion, round to nearest even)."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).view(np.uint16)
+
+
+# The eight timesteps of the distilled sampler (FastH3 Trim, "What Trim changes").
+SAMPLER_TIMESTEPS = (999, 874, 749, 624, 500, 375, 250, 125)
+
+
+def adaln_inputs(blocks: int, n: int, d: int, r: int, timesteps, seed: int = 0):
+    """Synthetic stand-ins for the AdaLN basis projection (no trained weights exist here):
+    time embeddings e [bt, d] BF16 ~ N(0, 1), one seeded row per timestep; shared basis
+    [r, d] FP16 ~ N(0, 1/d) (rows of about unit norm); per-block projections [blocks, n, r]
+    FP16 ~ N(0, 0.05^2); per-block biases [blocks, n] FP16 ~ N(0, 0.01^2)."""
+    e = np.stack([normal(derive_seed("temb", seed, int(t), d), 0, d) for t in timesteps]) if len(timesteps) \
+        else np.zeros((0, d))
+    basis = normal(derive_seed("adaln-basis", seed, r, d), 0, r * d).reshape(r, d) / np.sqrt(d)
+    proj = normal(derive_seed("adaln-proj", seed, blocks, n, r), 0, blocks * n * r).reshape(blocks, n, r) * 0.05
+    bias = normal(derive_seed("adaln-bias", seed, blocks, n), 0, blocks * n).reshape(blocks, n) * 0.01
+    return to_bf16_bits(e), to_f16_bits(basis), to_f16_bits(proj), to_f16_bits(bias)
