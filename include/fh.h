@@ -216,6 +216,27 @@ int fh_int8_attention_scores(const int8_t* q_dev, const float* q_scales_dev, con
                              const float* k_scales_dev, float sm_scale, float* s_dev, int64_t heads, int64_t tq,
                              int64_t tk, int64_t d, fh_stream_t stream);
 
+/* AdaLN timestep conditioning through a shared low-rank basis.  FastH3 Trim
+ * (comfyui-wiki news), "What Trim changes": AdaLN maps the 2,688-wide time
+ * embedding to six modulation vectors per block; Trim replaces the per-block
+ * projections with one shared 2,688 -> 16 basis and a small projection per
+ * block, stored in FP16.  This call evaluates both maps, linear, in FP32:
+ *   code[b, j]   = sum_k basis[j, k] * temb[b, k]
+ *   mod[l, b, i] = sum_j proj[l, i, j] * code[b, j] + bias[l, i]
+ * temb_dev: BF16 [bt, d]; basis_dev: FP16 [r, d]; proj_dev: FP16 [blocks, n, r];
+ * bias_dev: FP16 [blocks, n] or NULL (no bias); code_dev: FP32 [bt, r], written
+ * (the shared code, an output the caller owns); mod_dev: FP32 [blocks, bt, n],
+ * written (for the pages' model n = 6 * 2688, the six modulation vectors of a
+ * block side by side).  bt, blocks, n >= 0 (blocks * n < 2^31); d > 0,
+ * d % 8 == 0; r in {8, 16, 24, 32}; temb, basis and proj 16-byte aligned, bias
+ * 2-byte, code and mod 4-byte.  The result is within the FP32 dot-product bound
+ * of the exact value; it is exact when every partial sum is representable.
+ * Two kernels run on `stream`, the second launched as a programmatic
+ * dependent of the first. */
+int fh_adaln_modulation(const uint16_t* temb_dev, int64_t bt, int64_t d, const uint16_t* basis_dev, int64_t r,
+                        const uint16_t* proj_dev, const uint16_t* bias_dev, int64_t blocks, int64_t n,
+                        float* code_dev, float* mod_dev, fh_stream_t stream);
+
 /* Diagnostic of the failure path: enqueues a one-thread kernel whose bounded
  * mbarrier wait (the same wait every pipeline stage of fh_nvfp4_linear uses)
  * can never be satisfied and gives up after limit_us microseconds (1 .. 2e6),

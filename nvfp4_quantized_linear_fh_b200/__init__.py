@@ -62,6 +62,7 @@ _SIG = {
     "fh_gelu_bf16": (_c.c_int, [_P, _P, _I64, _P]),
     "fh_quantize_int8_rows": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fh_int8_attention_scores": (_c.c_int, [_P, _P, _P, _P, _c.c_float, _P, _I64, _I64, _I64, _I64, _P]),
+    "fh_adaln_modulation": (_c.c_int, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P]),
     "fh_device_status": (_c.c_int, [_P]),
     "fh_selftest_bounded_wait": (_c.c_int, [_c.c_uint32, _P]),
 }
@@ -277,6 +278,31 @@ def fh_int8_attention_scores(q: torch.Tensor, q_scales: torch.Tensor, k: torch.T
         raise ValueError("shape mismatch: q [H, tq, d], k [H, tk, d], scales [H, t], s [H, tq, tk]")
     _check(_lib.fh_int8_attention_scores(_ptr(q), _ptr(q_scales), _ptr(k), _ptr(k_scales), float(sm_scale),
                                          _ptr(s), heads, tq, tk, d, _stream(stream)))
+
+
+def fh_adaln_modulation(temb: torch.Tensor, basis: torch.Tensor, proj: torch.Tensor, bias: torch.Tensor | None,
+                        code: torch.Tensor, mod: torch.Tensor, stream=None) -> None:
+    """code [bt, r] = temb [bt, d] . basis^T (basis [r, d] FP16); mod [blocks, bt, n] = proj [blocks, n, r] . code^T
+    + bias [blocks, n], all FP32 results."""
+    _need(temb, _BF16, "temb", 2)
+    _need(basis, (torch.float16,), "basis", 2)
+    _need(proj, (torch.float16,), "proj", 3)
+    _need(code, (torch.float32,), "code", 2)
+    _need(mod, (torch.float32,), "mod", 3)
+    if bias is not None:
+        _need(bias, (torch.float16,), "bias", 2)
+    for t, nm in ((temb, "temb"), (basis, "basis"), (proj, "proj"), (code, "code"), (mod, "mod"), (bias, "bias")):
+        if t is not None and not t.is_contiguous():
+            raise ValueError(f"{nm} must be contiguous")
+    bt, d = temb.shape
+    r = basis.shape[0]
+    blocks, n = proj.shape[0], proj.shape[1]
+    if (basis.shape[1] != d or proj.shape[2] != r or tuple(code.shape) != (bt, r)
+            or tuple(mod.shape) != (blocks, bt, n) or (bias is not None and tuple(bias.shape) != (blocks, n))):
+        raise ValueError("shape mismatch: temb [bt, d], basis [r, d], proj [blocks, n, r], bias [blocks, n], "
+                         "code [bt, r], mod [blocks, bt, n]")
+    _check(_lib.fh_adaln_modulation(_ptr(temb), bt, d, _ptr(basis), r, _ptr(proj), _ptr(bias), blocks, n,
+                                    _ptr(code), _ptr(mod), _stream(stream)))
 
 
 def fh_selftest_bounded_wait(limit_us: int, stream=None) -> None:

@@ -280,6 +280,32 @@ int fh_int8_attention_scores(const int8_t* q_dev, const float* q_scales_dev, con
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_int8_attention_scores launch");
 }
 
+int fh_adaln_modulation(const uint16_t* temb_dev, int64_t bt, int64_t d, const uint16_t* basis_dev, int64_t r,
+                        const uint16_t* proj_dev, const uint16_t* bias_dev, int64_t blocks, int64_t n,
+                        float* code_dev, float* mod_dev, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (bt < 0 || d <= 0 || d % 8 != 0 || blocks < 0 || n < 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_adaln_modulation: need bt, blocks, n >= 0, d > 0, d %% 8 == 0%s");
+  if (r != 8 && r != 16 && r != 24 && r != 32)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_adaln_modulation: the basis rank r must be 8, 16, 24 or 32%s");
+  if (blocks * n > 0x7FFFFFFF || bt * r > ((int64_t)1 << 40) || d > ((int64_t)1 << 40))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_adaln_modulation: tensor too large%s");
+  if (bt == 0) return FH_OK;
+  if (temb_dev == nullptr || basis_dev == nullptr || code_dev == nullptr ||
+      (blocks * n > 0 && (proj_dev == nullptr || mod_dev == nullptr)))
+    return fail(FH_ERR_INVALID_ARG, "fh_adaln_modulation: null pointer%s");
+  if (!aligned16(temb_dev) || !aligned16(basis_dev) || (proj_dev != nullptr && !aligned16(proj_dev)) ||
+      (reinterpret_cast<uintptr_t>(bias_dev) & 1u) != 0 || (reinterpret_cast<uintptr_t>(code_dev) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(mod_dev) & 3u) != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_adaln_modulation: temb, basis and proj must be 16-byte aligned, bias 2-byte, code and mod "
+                "4-byte%s");
+  if (int st = check_device()) return st;
+  cudaError_t e = fh::launch_adaln_modulation(temb_dev, bt, d, basis_dev, r, proj_dev, bias_dev, blocks, n, code_dev,
+                                              mod_dev, (cudaStream_t)stream);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_adaln_modulation launch");
+}
+
 int fh_selftest_bounded_wait(uint32_t limit_us, fh_stream_t stream) {
   g_last_error[0] = 0;
   if (limit_us == 0 || limit_us > 2000000u)

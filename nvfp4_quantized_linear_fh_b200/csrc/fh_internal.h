@@ -85,4 +85,11 @@ cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int
                                float sm_scale, float* out, int64_t heads, int64_t tq, int64_t tk, int64_t d,
                                cudaStream_t s, const char** why);
 
+// AdaLN basis projection (fh_adaln.cu): code [bt, r] = e . basis^T, then
+// mod [L, bt, n] = proj . code^T + bias, in FP32 from BF16 e and FP16 weights.
+// r in {8, 16, 24, 32}; d % 8 == 0.  Arguments are validated by the caller.
+cudaError_t launch_adaln_modulation(const uint16_t* e, int64_t bt, int64_t d, const uint16_t* basis, int64_t r,
+                                    const uint16_t* proj, const uint16_t* bias, int64_t L, int64_t n, float* code,
+                                    float* mod, cudaStream_t s);
+
 }  // namespace fh

@@ -125,6 +125,15 @@ def test_argument_validation_without_gpu(lib):
     assert s(fake, fake, P(40), fake, 1.0, fake, 2, 100, 256, 128, None) == 2  # k misaligned
     assert s(fake, fake, fake, fake, 1.0, fake, 2, 0, 256, 128, None) == 0     # empty
     assert s(fake, fake, fake, fake, 1.0, fake, 0, 100, 256, 128, None) == 0
+    d = lib.fh_adaln_modulation
+    d.argtypes = [P, ctypes.c_int64, ctypes.c_int64, P, ctypes.c_int64, P, P, ctypes.c_int64, ctypes.c_int64, P, P, P]
+    assert d(fake, 8, 2688, fake, 12, fake, None, 42, 16128, fake, fake, None) == 2   # rank not in {8,16,24,32}
+    assert d(fake, 8, 2684, fake, 16, fake, None, 42, 16128, fake, fake, None) == 2   # d % 8
+    assert d(fake, 8, 2688, fake, 16, fake, None, 1 << 20, 1 << 12, fake, fake, None) == 2  # blocks * n >= 2^31
+    assert d(fake, 8, 2688, None, 16, fake, None, 42, 16128, fake, fake, None) == 1   # null basis
+    assert d(fake, 8, 2688, fake, 16, P(24), None, 42, 16128, fake, fake, None) == 2  # proj misaligned
+    assert d(fake, 8, 2688, fake, 16, fake, P(17), 42, 16128, fake, fake, None) == 2  # bias misaligned
+    assert d(fake, 0, 2688, fake, 16, fake, None, 42, 16128, fake, fake, None) == 0   # no timesteps
     a = lib.fh_amax
     a.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P]
     assert a(fake, 3, 5, 4, fake, None) == 2
