@@ -508,6 +508,105 @@ def bench_attn(args):
     print(json.dumps(line))
 
 
+ADALN = {"blocks": 42, "n": 6 * 2688, "d": 2688, "r": 16}
+
+
+def adaln_bytes(blocks, n, d, r, bt):
+    """Algorithmic bytes of one fh_adaln_modulation call: embeddings, basis, projections
+    and biases read once; codes and modulations written once."""
+    return 2 * bt * d + 2 * r * d + 2 * blocks * n * r + 2 * blocks * n + 4 * bt * r + 4 * blocks * bt * n
+
+
+def bench_adaln(args):
+    """AdaLN timestep conditioning of the 42-block pruned transformer: the eight
+    sampler timesteps' 2688-wide embeddings through the shared 2688->16 basis and
+    each block's 16->6*2688 projection (FP16 weights, FP32 results).  The inputs
+    (45 MB) fit in L2, so L2 is flushed (a 256 MB write) before every timed call."""
+    import torch
+    import synthetic as S
+    import nvfp4_quantized_linear_fh_b200 as fh
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L, n, d, r = ADALN["blocks"], ADALN["n"], ADALN["d"], ADALN["r"]
+    ts = S.SAMPLER_TIMESTEPS
+    bt = len(ts)
+    e_b, basis_b, proj_b, bias_b = S.adaln_inputs(L, n, d, r, ts)
+
+    def to_dev(bits, dtype):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(dtype)
+
+    e, basis = to_dev(e_b, torch.bfloat16), to_dev(basis_b, torch.float16)
+    proj, bias = to_dev(proj_b, torch.float16), to_dev(bias_b, torch.float16)
+    code = torch.empty((bt, r), dtype=torch.float32, device=dev)
+    mod = torch.empty((L, bt, n), dtype=torch.float32, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MB > L2
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        fh.fh_adaln_modulation(e, basis, proj, bias, code, mod)
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 500))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    sampler = ClockSampler(f"GPU-{torch.cuda.get_device_properties(dev).uuid}")
+    with sampler:
+        sampler.wait_first_sample()
+        sampler.mark_start()
+        for i in range(steps):
+            flush.fill_(float(i))
+            ev[i][0].record(stream)
+            fh.fh_adaln_modulation(e, basis, proj, bias, code, mod)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        sampler.mark_end()
+    fh.fh_device_status()
+    t = sum(ev[i][0].elapsed_time(ev[i][1]) for i in range(steps)) * 1e-3 / steps
+    by = adaln_bytes(L, n, d, r, bt)
+
+    t_e2e, e_steps = float("nan"), 0
+    if not args.no_e2e:
+        e_h = torch.empty(e.shape, dtype=torch.bfloat16).pin_memory()
+        e_h.copy_(e.cpu())
+        mod_h = torch.empty(mod.shape, dtype=torch.float32).pin_memory()
+        e_steps = 20
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(e_steps):
+            e.copy_(e_h, non_blocking=True)
+            fh.fh_adaln_modulation(e, basis, proj, bias, code, mod)
+            mod_h.copy_(mod, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t_e2e = e0.elapsed_time(e1) * 1e-3 / e_steps
+
+    pk = peaks()
+    line = {
+        "metric": "AdaLN basis projection: GB/s of algorithmic HBM traffic per call (8 timesteps x 42 blocks)",
+        "value": by / t / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (FP16 weights, BF16 embeddings)", "data": "synthetic (seeded; random-init weights)",
+        "config": {"workload": f"AdaLN modulation {bt} timesteps x {L} blocks x {n} (d {d}, rank {r})",
+                   "blocks": L, "n": n, "d": d, "r": r, "timesteps": bt,
+                   "l2": "flushed before every timed call (256 MB write, outside the timed events)"},
+        "roofline": {"bound": "hbm", "kernel": "adaln_code_kernel + adaln_mod_kernel (one call)",
+                     "achieved": by / t / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": by / t / 1e9 / pk["hbm_gbs"], "peak_source": pk["source"], "traffic": None,
+                     "algorithmic_bytes": by},
+        "e2e": {"value": by / t_e2e / 1e9 if e_steps else None, "unit": "GB/s",
+                "h2d_bytes_per_step": 2 * bt * d, "d2h_bytes_per_step": 4 * L * bt * n},
+        "gpu_launches": 2 * steps, "clocks": sampler.summary(),
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        t0 = time.perf_counter()
+        for _ in range(3):
+            oracle.adaln_modulation(oracle.adaln_code(e_b, basis_b), proj_b, bias_b)
+        dt = (time.perf_counter() - t0) / 3
+        line["cpu_baseline"] = {"value": by / dt / 1e9, "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
+                                "kind": "oracle", "sample": "the whole call (8 timesteps, 42 blocks), 3 runs"}
+    print(json.dumps(line))
+
+
 # DRAM bytes (read + write) of one int8_scores_kernel launch on the workload
 # above, from an ncu capture; valid only for the kernel source it was taken on.
 ATTN_TRAFFIC = {"bytes": 1375100160, "source_sha256": "0630d6dd00149ba6"}
@@ -533,9 +632,10 @@ def main():
     ap.add_argument("--M", type=int, default=WORKLOAD["M"],
                     help="token rows per GPU (profiling cases use fewer than the workload's 32768)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
-    ap.add_argument("--workload", default="qkv", choices=["qkv", "ffn", "attn"],
+    ap.add_argument("--workload", default="qkv", choices=["qkv", "ffn", "attn", "adaln"],
                     help="qkv: the headline line (fused QKV layer); ffn: the FFN block, fused vs unfused "
-                         "epilogue; attn: INT8 query/key quantization and attention scores")
+                         "epilogue; attn: INT8 query/key quantization and attention scores; adaln: AdaLN "
+                         "basis projection")
     ap.add_argument("--quick", action="store_true",
                     help="calibrate on the input batches only (setup shortcut for profiling cases)")
     args = ap.parse_args()
@@ -545,6 +645,9 @@ def main():
         return
     if args.workload == "attn":
         bench_attn(args)
+        return
+    if args.workload == "adaln":
+        bench_adaln(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -8,14 +8,18 @@
 //   mod[l, b, i] = sum_j proj[l, i, j] code[b, j] + bias[l, i]      (FP32)
 //
 // Two kernels, chained by programmatic dependent launch:
-//   adaln_code_kernel  one warp per (b, j): a 16-byte-load dot product over d.
-//                      It lets the dependent grid start at once.
-//   adaln_mod_kernel   one thread per (l, i): its r FP16 weights and its bias
-//                      are loaded into registers before griddepcontrol.wait, so
-//                      that the HBM read of the projections overlaps the code
-//                      kernel; then the codes are staged in shared memory (128
-//                      timesteps at a time) and each timestep's row of
-//                      modulations is written with coalesced FP32 stores.
+//   adaln_code_kernel  one CTA per (b, four basis rows): independent 16-byte
+//                      loads across the CTA, then a block reduction.  It lets
+//                      the dependent grid start at once.
+//   adaln_mod_kernel   one resident wave of CTAs walking groups of projection
+//                      rows (two per thread); each thread's FP16 rows and
+//                      biases for the first group are read before
+//                      griddepcontrol.wait, so that this HBM read overlaps the
+//                      code kernel, and the next group's are in flight while
+//                      the current one is computed.  The codes are staged in
+//                      shared memory once per CTA (128 timesteps at a time) and
+//                      each timestep's row of modulations is written with
+//                      coalesced FP32 stores.
 // The work is HBM-bound: the projections are read once, the modulations
 // written once.  Neither kernel waits on anything it must bound.
 #include <cuda_fp16.h>
@@ -37,87 +41,128 @@ __device__ __forceinline__ float2 half2_to_float2(uint32_t w) {
   return __half22float2(h);
 }
 
-// code [bt, r] = e [bt, d] . basis^T, basis [r, d]; d % 8 == 0.
-__global__ void __launch_bounds__(256) adaln_code_kernel(const uint16_t* __restrict__ e, int64_t bt, int64_t d,
-                                                         const uint16_t* __restrict__ basis, int r,
-                                                         float* __restrict__ code) {
+// code [bt, r] = e [bt, d] . basis^T, basis [r, d]; d % 8 == 0.  Block (b, g)
+// computes code[b, 4g .. 4g+3]: every thread loads its 16-byte chunks of the
+// embedding row and of the four basis rows at once (no dependent loads), then
+// the block reduces the four partial sums.
+constexpr int kCodeThreads = 256;
+__global__ void __launch_bounds__(kCodeThreads) adaln_code_kernel(const uint16_t* __restrict__ e, int64_t d,
+                                                                  const uint16_t* __restrict__ basis, int r,
+                                                                  float* __restrict__ code) {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  const int lane = threadIdx.x & 31;
-  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < bt * r; w += warps) {
-    const int64_t b = w / r;
-    const int j = (int)(w % r);
-    const uint16_t* er = e + b * d;
-    const uint16_t* br = basis + (int64_t)j * d;
-    float acc = 0.0f;
-    for (int64_t c = 8 * lane; c < d; c += 256) {
-      const uint4 ev = *reinterpret_cast<const uint4*>(er + c);
-      const uint4 bv = *reinterpret_cast<const uint4*>(br + c);
-      const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
-      const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+  __shared__ float part[kCodeThreads / 32][4];
+  const int64_t b = blockIdx.x;
+  const int j0 = 4 * blockIdx.y;
+  const uint16_t* er = e + b * d;
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int64_t c = 8 * (int64_t)threadIdx.x; c < d; c += 8 * kCodeThreads) {
+    const uint4 ev = *reinterpret_cast<const uint4*>(er + c);
+    uint4 bv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) bv[q] = *reinterpret_cast<const uint4*>(basis + (int64_t)(j0 + q) * d + c);
+    const uint32_t ew[4] = {ev.x, ev.y, ev.z, ev.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t bw[4] = {bv[q].x, bv[q].y, bv[q].z, bv[q].w};
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const float2 bf = half2_to_float2(bw[k]);
-        acc = fmaf(bf16_lo(ew[k]), bf.x, acc);
-        acc = fmaf(bf16_hi(ew[k]), bf.y, acc);
+        acc[q] = fmaf(bf16_lo(ew[k]), bf.x, acc[q]);
+        acc[q] = fmaf(bf16_hi(ew[k]), bf.y, acc[q]);
       }
     }
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
-    if (lane == 0) code[w] = acc;
+  for (int q = 0; q < 4; ++q) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[q] += __shfl_xor_sync(0xFFFFFFFFu, acc[q], o);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) part[warp][q] = acc[q];
+  }
+  __syncthreads();
+  if (threadIdx.x < 4) {
+    float t = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kCodeThreads / 32; ++w) t += part[w][threadIdx.x];
+    code[b * r + j0 + threadIdx.x] = t;
   }
 }
 
 constexpr int kCodeRows = 128;  // timesteps whose codes are staged in shared memory at once
+constexpr int kModThreads = 256;
+constexpr int kModRows = 2;     // projection rows per thread per group
 
 // mod [L, bt, n] = proj [L, n, r] . code [bt, r]^T + bias [L, n]; r = 8 * RC.
+// Row groups of kModThreads * kModRows rows are walked grid-stride; a thread
+// holds the raw FP16 rows of its current group and has the next group's in
+// flight.  The first group is loaded before griddepcontrol.wait.
 template <int RC>
-__global__ void __launch_bounds__(256) adaln_mod_kernel(const uint16_t* __restrict__ proj,
-                                                        const uint16_t* __restrict__ bias,
-                                                        const float* __restrict__ code, int64_t bt, int64_t L,
-                                                        int64_t n, float* __restrict__ mod) {
+__global__ void __launch_bounds__(kModThreads) adaln_mod_kernel(const uint16_t* __restrict__ proj,
+                                                                const uint16_t* __restrict__ bias,
+                                                                const float* __restrict__ code, int64_t bt,
+                                                                int64_t rows_total, int64_t n,
+                                                                float* __restrict__ mod) {
   constexpr int R = 8 * RC;
+  constexpr int64_t kGroup = (int64_t)kModThreads * kModRows;
   __shared__ float code_s[kCodeRows * R];
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const bool live = idx < L * n;
-  const int64_t l = live ? idx / n : 0, i = live ? idx % n : 0;
-  // The projection row and bias do not depend on the code kernel: load them first.
-  float p[R];
-  float c0 = 0.0f;
-  if (live) {
-    const uint4* pr = reinterpret_cast<const uint4*>(proj + idx * R);
+  struct Raw {
+    uint4 w[kModRows][RC];
+    uint16_t c[kModRows];
+  };
+  auto fetch = [&](int64_t g, Raw& raw) {
 #pragma unroll
-    for (int q = 0; q < RC; ++q) {
-      const uint4 v = pr[q];
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int k = 0; k < kModRows; ++k) {
+      const int64_t idx = g * kGroup + (int64_t)k * kModThreads + threadIdx.x;
+      const bool live = idx < rows_total;
+      const uint4* pr = reinterpret_cast<const uint4*>(proj + (live ? idx : 0) * R);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 f = half2_to_float2(w[k]);
-        p[8 * q + 2 * k] = f.x;
-        p[8 * q + 2 * k + 1] = f.y;
-      }
+      for (int q = 0; q < RC; ++q) raw.w[k][q] = live ? pr[q] : make_uint4(0, 0, 0, 0);
+      raw.c[k] = (live && bias != nullptr) ? bias[idx] : (uint16_t)0;
     }
-    if (bias != nullptr) c0 = __half2float(__ushort_as_half(bias[idx]));
-  } else {
-#pragma unroll
-    for (int j = 0; j < R; ++j) p[j] = 0.0f;
-  }
-  // The codes are written by the preceding grid.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  };
+  const int64_t groups = (rows_total + kGroup - 1) / kGroup;
+  Raw cur, nxt;
+  // The projections do not depend on the code kernel: start reading them now.
+  if ((int64_t)blockIdx.x < groups) fetch(blockIdx.x, cur);
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the codes are written by the preceding grid
   for (int64_t b0 = 0; b0 < bt; b0 += kCodeRows) {
-    const int rows = (int)(bt - b0 < kCodeRows ? bt - b0 : kCodeRows);
+    const int nb = (int)(bt - b0 < kCodeRows ? bt - b0 : kCodeRows);
     __syncthreads();  // the previous chunk's codes are no longer read
-    for (int t = threadIdx.x; t < rows * R; t += blockDim.x) code_s[t] = code[b0 * R + t];
+    for (int t = threadIdx.x; t < nb * R; t += kModThreads) code_s[t] = code[b0 * R + t];
     __syncthreads();
-    if (live) {
-      float* out = mod + (l * bt + b0) * n + i;
-      for (int b = 0; b < rows; ++b) {
-        const float* z = code_s + b * R;
-        float acc = c0;
+    if (b0 > 0 && (int64_t)blockIdx.x < groups) fetch(blockIdx.x, cur);  // later chunks re-read (from L2)
+    for (int64_t g = blockIdx.x; g < groups; g += gridDim.x) {
+      if (g + gridDim.x < groups) fetch(g + gridDim.x, nxt);
 #pragma unroll
-        for (int j = 0; j < R; ++j) acc = fmaf(p[j], z[j], acc);
-        out[(int64_t)b * n] = acc;
+      for (int k = 0; k < kModRows; ++k) {
+        const int64_t idx = g * kGroup + (int64_t)k * kModThreads + threadIdx.x;
+        if (idx >= rows_total) continue;
+        float p[R];
+#pragma unroll
+        for (int q = 0; q < RC; ++q) {
+          const uint32_t w[4] = {cur.w[k][q].x, cur.w[k][q].y, cur.w[k][q].z, cur.w[k][q].w};
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 f = half2_to_float2(w[h]);
+            p[8 * q + 2 * h] = f.x;
+            p[8 * q + 2 * h + 1] = f.y;
+          }
+        }
+        const float c0 = __half2float(__ushort_as_half(cur.c[k]));
+        const int64_t l = idx / n, i = idx % n;
+        float* out = mod + (l * bt + b0) * n + i;
+        for (int b = 0; b < nb; ++b) {
+          const float* z = code_s + b * R;
+          float acc = c0;
+#pragma unroll
+          for (int j = 0; j < R; ++j) acc = fmaf(p[j], z[j], acc);
+          out[(int64_t)b * n] = acc;
+        }
       }
+      cur = nxt;
     }
   }
 }
@@ -125,10 +170,18 @@ __global__ void __launch_bounds__(256) adaln_mod_kernel(const uint16_t* __restri
 template <int RC>
 cudaError_t launch_mod(const uint16_t* proj, const uint16_t* bias, const float* code, int64_t bt, int64_t L,
                        int64_t n, float* mod, cudaStream_t s) {
-  const int64_t threads = L * n;
+  const int64_t rows_total = L * n;
+  const int64_t groups = (rows_total + (int64_t)kModThreads * kModRows - 1) / ((int64_t)kModThreads * kModRows);
+  static int per_sm = 0;  // resident CTAs per SM for this instantiation (one wave)
+  if (per_sm == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_mod_kernel<RC>, kModThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+  }
+  const int64_t cap = (int64_t)sm_count() * per_sm;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((threads + 255) / 256));
-  cfg.blockDim = dim3(256);
+  cfg.gridDim = dim3((unsigned)(groups < cap ? groups : cap));
+  cfg.blockDim = dim3(kModThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -136,7 +189,7 @@ cudaError_t launch_mod(const uint16_t* proj, const uint16_t* bias, const float* 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, adaln_mod_kernel<RC>, proj, bias, code, bt, L, n, mod);
+  return cudaLaunchKernelEx(&cfg, adaln_mod_kernel<RC>, proj, bias, code, bt, rows_total, n, mod);
 }
 
 }  // namespace
@@ -144,11 +197,7 @@ cudaError_t launch_mod(const uint16_t* proj, const uint16_t* bias, const float* 
 cudaError_t launch_adaln_modulation(const uint16_t* e, int64_t bt, int64_t d, const uint16_t* basis, int64_t r,
                                     const uint16_t* proj, const uint16_t* bias, int64_t L, int64_t n, float* code,
                                     float* mod, cudaStream_t s) {
-  const int64_t warps_needed = bt * r;
-  const int64_t cap = (int64_t)sm_count() * 8;
-  const int64_t blocks = (warps_needed + 7) / 8;
-  const int grid = (int)(blocks < cap ? (blocks > 0 ? blocks : 1) : cap);
-  adaln_code_kernel<<<grid, 256, 0, s>>>(e, bt, d, basis, (int)r, code);
+  adaln_code_kernel<<<dim3((unsigned)bt, (unsigned)(r / 4)), kCodeThreads, 0, s>>>(e, d, basis, (int)r, code);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   if (L * n == 0) return cudaSuccess;  // only the codes were asked for

@@ -288,7 +288,7 @@ int fh_adaln_modulation(const uint16_t* temb_dev, int64_t bt, int64_t d, const u
     return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_adaln_modulation: need bt, blocks, n >= 0, d > 0, d %% 8 == 0%s");
   if (r != 8 && r != 16 && r != 24 && r != 32)
     return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_adaln_modulation: the basis rank r must be 8, 16, 24 or 32%s");
-  if (blocks * n > 0x7FFFFFFF || bt * r > ((int64_t)1 << 40) || d > ((int64_t)1 << 40))
+  if (blocks * n > 0x7FFFFFFF || bt > 0x7FFFFFFF || d > ((int64_t)1 << 40))
     return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_adaln_modulation: tensor too large%s");
   if (bt == 0) return FH_OK;
   if (temb_dev == nullptr || basis_dev == nullptr || code_dev == nullptr ||
