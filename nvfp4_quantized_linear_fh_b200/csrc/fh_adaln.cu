@@ -17,9 +17,11 @@
 //                      griddepcontrol.wait, so that this HBM read overlaps the
 //                      code kernel, and the next group's are in flight while
 //                      the current one is computed.  The codes are staged in
-//                      shared memory once per CTA (128 timesteps at a time) and
-//                      each timestep's row of modulations is written with
-//                      coalesced FP32 stores.
+//                      shared memory once per CTA (128 timesteps at a time),
+//                      interleaved by timestep pairs so that packed FP32 FMAs
+//                      evaluate two timesteps per instruction, and each
+//                      timestep's row of modulations is written with coalesced
+//                      FP32 stores.
 // The work is HBM-bound: the projections are read once, the modulations
 // written once.  Neither kernel waits on anything it must bound.
 #include <cuda_fp16.h>
@@ -107,7 +109,9 @@ __global__ void __launch_bounds__(kModThreads) adaln_mod_kernel(const uint16_t* 
                                                                 float* __restrict__ mod) {
   constexpr int R = 8 * RC;
   constexpr int64_t kGroup = (int64_t)kModThreads * kModRows;
-  __shared__ float code_s[kCodeRows * R];
+  // Codes of timestep pairs interleaved, [b / 2][j][b % 2], so that one 16-byte
+  // load gives (z[b][j], z[b+1][j], z[b][j+1], z[b+1][j+1]) for packed FMAs.
+  __shared__ float4 code_s[kCodeRows / 2 * R / 2];
   struct Raw {
     uint4 w[kModRows][RC];
     uint16_t c[kModRows];
@@ -130,36 +134,60 @@ __global__ void __launch_bounds__(kModThreads) adaln_mod_kernel(const uint16_t* 
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the codes are written by the preceding grid
   for (int64_t b0 = 0; b0 < bt; b0 += kCodeRows) {
     const int nb = (int)(bt - b0 < kCodeRows ? bt - b0 : kCodeRows);
+    const int npairs = (nb + 1) / 2;
     __syncthreads();  // the previous chunk's codes are no longer read
-    for (int t = threadIdx.x; t < nb * R; t += kModThreads) code_s[t] = code[b0 * R + t];
+    float* cs = reinterpret_cast<float*>(code_s);
+    for (int t = threadIdx.x; t < npairs * 2 * R; t += kModThreads) {
+      const int bb = 2 * (t / (2 * R)) + (t & 1), j = (t % (2 * R)) >> 1;
+      cs[t] = bb < nb ? code[(b0 + bb) * R + j] : 0.0f;  // an odd count pads with zeros
+    }
     __syncthreads();
     if (b0 > 0 && (int64_t)blockIdx.x < groups) fetch(blockIdx.x, cur);  // later chunks re-read (from L2)
     for (int64_t g = blockIdx.x; g < groups; g += gridDim.x) {
       if (g + gridDim.x < groups) fetch(g + gridDim.x, nxt);
+      float2 pp[kModRows][R];  // (p_j, p_j): the weight against both timesteps of a pair
+      float2 c2[kModRows];
+      float* out[kModRows];
+      bool live[kModRows];
 #pragma unroll
       for (int k = 0; k < kModRows; ++k) {
         const int64_t idx = g * kGroup + (int64_t)k * kModThreads + threadIdx.x;
-        if (idx >= rows_total) continue;
-        float p[R];
+        live[k] = idx < rows_total;
 #pragma unroll
         for (int q = 0; q < RC; ++q) {
           const uint32_t w[4] = {cur.w[k][q].x, cur.w[k][q].y, cur.w[k][q].z, cur.w[k][q].w};
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             const float2 f = half2_to_float2(w[h]);
-            p[8 * q + 2 * h] = f.x;
-            p[8 * q + 2 * h + 1] = f.y;
+            pp[k][8 * q + 2 * h] = make_float2(f.x, f.x);
+            pp[k][8 * q + 2 * h + 1] = make_float2(f.y, f.y);
           }
         }
         const float c0 = __half2float(__ushort_as_half(cur.c[k]));
-        const int64_t l = idx / n, i = idx % n;
-        float* out = mod + (l * bt + b0) * n + i;
-        for (int b = 0; b < nb; ++b) {
-          const float* z = code_s + b * R;
-          float acc = c0;
+        c2[k] = make_float2(c0, c0);
+        const uint32_t row = live[k] ? (uint32_t)idx : 0u;  // rows_total < 2^31
+        const uint32_t l = row / (uint32_t)n, i = row - l * (uint32_t)n;
+        out[k] = mod + ((int64_t)l * bt + b0) * n + i;
+      }
+      for (int bp = 0; bp < npairs; ++bp) {
+        float2 acc[kModRows];
 #pragma unroll
-          for (int j = 0; j < R; ++j) acc = fmaf(p[j], z[j], acc);
-          out[(int64_t)b * n] = acc;
+        for (int k = 0; k < kModRows; ++k) acc[k] = c2[k];
+#pragma unroll
+        for (int jq = 0; jq < R / 2; ++jq) {
+          const float4 zz = code_s[bp * (R / 2) + jq];
+#pragma unroll
+          for (int k = 0; k < kModRows; ++k) {
+            acc[k] = __ffma2_rn(pp[k][2 * jq], make_float2(zz.x, zz.y), acc[k]);
+            acc[k] = __ffma2_rn(pp[k][2 * jq + 1], make_float2(zz.z, zz.w), acc[k]);
+          }
+        }
+        const int b = 2 * bp;
+#pragma unroll
+        for (int k = 0; k < kModRows; ++k) {
+          if (!live[k]) continue;
+          out[k][(int64_t)b * n] = acc[k].x;
+          if (b + 1 < nb) out[k][(int64_t)(b + 1) * n] = acc[k].y;
         }
       }
       cur = nxt;
