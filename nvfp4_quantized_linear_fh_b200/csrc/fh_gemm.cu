@@ -12,31 +12,33 @@
 // cta_group::2 (each SM computes 128 rows; the 192 W rows are split 96/96
 // between the two SMs' shared memory, so each SM loads and holds half of W);
 // the single-CTA form (128 x 192 tiles) is the same code with kCta = 1.
-// Per CTA, 320 threads:
-//   warp 0      TMA producer: per 256-wide K stage, its 128 x 128-byte A tile
-//               and its (192 / kCta) x 128-byte W tile (128-byte swizzle) by
-//               tensor TMA completing on the leader CTA's stage barrier, and the
-//               stage's scale atoms (512 bytes = 128 rows x 64 K) by bulk copies
-//               completing on a barrier of its own CTA.
+// Per CTA, 192 threads:
+//   warp 0      TMA producer: per 256-wide K stage, its 128 x 128-byte A tile,
+//               its (192 / kCta) x 128-byte W tile (128-byte swizzle), and the
+//               stage's scale atoms (512 bytes = 128 rows x 64 K; one box for
+//               this CTA's A rows, one for the tile's two W scale blocks), all
+//               by tensor TMA completing on the leader CTA's stage barrier.
 //   warp 1      allocates TMEM (512 columns, both CTAs); in the leader CTA one
-//               lane issues four tcgen05.mma kind::mxf4nvf4 block_scale
-//               (M = 128 kCta, N = 192, K = 64) per stage into one of two TMEM
-//               accumulators; tcgen05.commit (multicast to the pair) frees the
-//               stage's shared memory and scale buffer and, after the last
-//               stage, hands the accumulator to both CTAs' epilogues.
-//   warps 6..9  scale stagers, one per TMEM lane quadrant: copy the stage's
-//               scale atoms from shared memory into a 3-deep ring of TMEM scale
-//               buffers with tcgen05.st (each warp fills its own 32 lanes, which
-//               is the replication the MMA reads).  Moving the scales this way
-//               keeps them off the tensor pipe: tcgen05.cp of the same bytes
-//               serializes with the MMAs and would halve their rate.
+//               lane copies the stage's scale atoms from shared memory into one
+//               of two TMEM scale buffers (tcgen05.cp 32x128b.warpx4, which
+//               replicates each atom into the four lane quadrants, in both CTAs
+//               of the pair) and then issues four tcgen05.mma kind::mxf4nvf4
+//               block_scale (M = 128 kCta, N = 192, K = 64) into one of two TMEM
+//               accumulators.  Copies and MMAs run in issue order on the tensor
+//               pipe, so a scale buffer needs no barrier; double buffering
+//               keeps a copy from waiting on the MMAs still reading the other.
+//               tcgen05.commit (multicast to the pair) frees the stage's shared
+//               memory and, after the last stage, hands the accumulator to both
+//               CTAs' epilogues.
 //   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, alpha * acc + bias
 //               in FP32, BF16 round-to-nearest-even, 128-byte-swizzled staging
 //               in shared memory and TMA stores, while the MMA warp already fills
 //               the other accumulator.
-// TMEM columns (each CTA): accumulators [0, 192) and [192, 384); three scale
-// buffers of 40 columns from 384: per K=64 step, 4 columns of A scales (row r
-// at lane r%32, column r/32) then 6 columns of W scales for the tile's 192 rows.
+// TMEM columns (each CTA): accumulators [0, 192) and [192, 384); two scale
+// buffers of 48 columns from 384: per K=64 step, 4 columns of A scales (row r
+// at lane r%32, column r/32) then 8 columns of W scales (the two 128-row scale
+// blocks the tile's 192 rows fall in; the MMA reads 6 of them from column 0 or
+// 2).
 // No TMA load uses cluster multicast; only tcgen05.commit is multicast.
 // Every mbarrier wait is bounded; on expiry the kernel sets the device error
 // word, stops issuing work, drains what it issued and frees its TMEM.
@@ -64,15 +66,13 @@ constexpr int kABytes = 128 * BK / 2;    // 16384: one CTA's 128 A rows
 constexpr int kSFABytes = kKSteps * kAtomBytes;      // 2048
 constexpr int kSFBBytes = 2 * kKSteps * kAtomBytes;  // 4096
 constexpr int kEpiWarps = 4;
-constexpr int kSfWarps = 4;
 constexpr int kEpiCols = 64;                          // columns per TMA store box
 constexpr int kEpiBufBytes = 32 * kEpiCols * 2;       // 4096: 32 rows x 128 bytes
-constexpr int kThreads = 64 + 32 * (kEpiWarps + kSfWarps);  // 320
-constexpr int kFirstSfWarp = 2 + kEpiWarps;           // 6
+constexpr int kThreads = 64 + 32 * kEpiWarps;         // 192
 constexpr int kTmemCols = 512;
 constexpr int kAccCols = BN;
-constexpr int kSfCols = 4 * kKSteps + 6 * kKSteps;    // 40 per stage: A 4, W 6 per K=64 step
-constexpr int kSfBufs = 3;
+constexpr int kSfCols = 4 * kKSteps + 8 * kKSteps;    // 48 per stage: A 4, W 8 per K=64 step
+constexpr int kSfBufs = 2;
 constexpr int kSfCol0 = 2 * kAccCols;                 // 384
 static_assert(kSfCol0 + kSfBufs * kSfCols <= kTmemCols, "TMEM budget");
 
@@ -90,9 +90,8 @@ struct Cfg {
   static constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
   static constexpr int kOffBias = kOffEpi + kEpiWarps * kEpiBufs * kEpiBufBytes;
   static constexpr int kOffBar = kOffBias + kEpiWarps * BN * 4;
-  // full, empty, scale-smem (per stage); acc full, acc empty (x2); scale full,
-  // scale empty (x3); drain
-  static constexpr int kNumBars = 3 * kStages + 4 + 2 * kSfBufs + 1;
+  // full, empty (per stage); acc full, acc empty (x2); drain
+  static constexpr int kNumBars = 2 * kStages + 4 + 1;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
   // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1
@@ -106,16 +105,11 @@ struct Cfg {
 };
 
 struct Params {
-  const uint8_t* sfa;
-  const uint8_t* sfb;
   const uint16_t* bias;
   float alpha;
   int M, N, K;
   int n_tiles, num_tiles, k_stages;
   int ksteps_total;  // K / 64
-  int sf_katoms;     // K / 64: 512-byte atoms per 128-row scale block
-  int n_sfa_blocks;  // ceil(M / 128)
-  int n_sfb_blocks;  // ceil(N / 128)
   int stall_group;   // test hook: this CTA group's MMA warp stops after 3 stages (-1: none)
 };
 
@@ -292,15 +286,6 @@ __device__ __forceinline__ void arrive_expect_tx_leader(uint32_t bar, uint32_t b
     mbar_arrive_expect_tx(bar, bytes);
 }
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst),
-      "l"(src), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
@@ -383,6 +368,18 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
   }
 }
 
+// Copy one 512-byte scale atom (32 rows of 16 bytes: rows r, r+32, r+64, r+96
+// at row r) into four TMEM columns, replicated into all four lane quadrants --
+// the layout the block-scaled MMA reads.  kCta == 2: in both CTAs of the pair,
+// each from its own shared memory at the same offset.
+template <int kCta>
+__device__ __forceinline__ void tc_cp_atom(uint32_t taddr, uint64_t sdesc) {
+  if (kCta == 1)
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+  else
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 // 32 consecutive TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld_32(uint32_t taddr, uint32_t (&v)[32]) {
   asm volatile(
@@ -399,32 +396,6 @@ __device__ __forceinline__ void tmem_ld_32(uint32_t taddr, uint32_t (&v)[32]) {
 
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// 16 / 8 consecutive TMEM columns of this thread's lane from registers.
-__device__ __forceinline__ void tmem_st_16(uint32_t taddr, const uint32_t (&v)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
-      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_8(uint32_t taddr, const uint32_t (&v)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-               "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_st_wait() {
-  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint4 lds128(uint32_t addr) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-  return v;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -450,6 +421,7 @@ struct Ring {
 template <int kCta, int kEpi>
 __global__ void __launch_bounds__(kThreads, 1)
     nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                         const __grid_constant__ CUtensorMap tmY, const Params p,
                         const __grid_constant__ typename EpiSel<kEpi>::type eq) {
   using C = Cfg<kCta>;
@@ -459,14 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + C::kOffBar;
-  auto full_bar = [&](int s) { return bar0 + 8u * s; };            // leader: A and W landed (both CTAs)
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };            // leader: A, W and scales landed (both CTAs)
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };     // each CTA: stage free again
-  auto sfs_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };   // each CTA: its scale atoms landed
-  auto accf_bar = [&](int a) { return bar0 + 8u * (3 * S + a); };  // each CTA: accumulator ready
-  auto acce_bar = [&](int a) { return bar0 + 8u * (3 * S + 2 + a); };        // leader: accumulator drained
-  auto sff_bar = [&](int b) { return bar0 + 8u * (3 * S + 4 + b); };         // leader: scales staged
-  auto sfe_bar = [&](int b) { return bar0 + 8u * (3 * S + 4 + kSfBufs + b); };  // each CTA: scale buffer free
-  const uint32_t drain_bar = bar0 + 8u * (3 * S + 4 + 2 * kSfBufs);
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };  // each CTA: accumulator ready
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };  // leader: accumulator drained
+  const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kNumBars * 8);
   if constexpr (kEpi == 1) {
     // The next layer's decision table, in the (otherwise unused) output staging area.
@@ -488,21 +457,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < S; ++s) {
       mbar_init(full_bar(s), kCta);
       mbar_init(empty_bar(s), 1);
-      mbar_init(sfs_bar(s), 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(accf_bar(a), 1);
       mbar_init(acce_bar(a), kEpiWarps * kCta);
-    }
-    for (int b = 0; b < kSfBufs; ++b) {
-      mbar_init(sff_bar(b), kSfWarps * kCta);
-      mbar_init(sfe_bar(b), 1);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmSA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmSB)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmY)) : "memory");
   }
   if (warp == 1) {
@@ -532,42 +498,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int arow = m_tile * C::BM + (int)rank * 128;   // this CTA's A rows
         const int n0 = n_tile * BN;
         const int brow = n0 + (int)rank * C::kBRows;          // this CTA's W rows
-        const int ablk = arow / 128;
-        const bool has_sfa = ablk < p.n_sfa_blocks;
-        const int jb0 = n0 / 128;
-        const int nsfb = (jb0 + 1 < p.n_sfb_blocks) ? 2 : 1;
+        const int ablk = arow / 128;  // this CTA's scale block of A
+        const int jb0 = n0 / 128;      // first of the tile's two scale blocks of W
         for (int kt = 0; kt < p.k_stages; ++kt) {
           if (!__all_sync(0xFFFFFFFFu, wait_bounded(empty_bar(st.slot), st.phase ^ 1u, abort_flag))) {
             ok = false;
             break;
           }
-          const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
-          const uint32_t sf_bytes = (uint32_t)ks * kAtomBytes;
           const uint32_t fb = leader_bar<kCta>(full_bar(st.slot));
-          const uint32_t sb = sfs_bar(st.slot);
-          const size_t katom0 = (size_t)kt * kKSteps;
+          // Scale atoms: one 2048-byte box (the stage's four K=64 atoms, 8-byte
+          // elements) of this CTA's A scale block and of the tile's two W scale
+          // blocks; blocks and atoms past the arrays read as zero.
+          const int sx = kt * kKSteps * (kAtomBytes / 8);
           if (elect_one()) {
-            arrive_expect_tx_leader<kCta>(fb, kABytes + C::kBBytes);
+            arrive_expect_tx_leader<kCta>(fb, kABytes + C::kBBytes + kSFABytes + kSFBBytes);
             tma_load_2d<kCta>(sbase + C::kOffA + st.slot * kABytes, &tmA, fb, kt * (BK / 2), arow);
             tma_load_2d<kCta>(sbase + C::kOffB + st.slot * C::kBBytes, &tmB, fb, kt * (BK / 2), brow);
-            mbar_arrive_expect_tx(sb, sf_bytes * ((has_sfa ? 1u : 0u) + (uint32_t)nsfb));
-            if (has_sfa)
-              bulk_load(sbase + C::kOffSFA + st.slot * kSFABytes,
-                        p.sfa + ((size_t)ablk * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
-            for (int r = 0; r < nsfb; ++r)
-              bulk_load(sbase + C::kOffSFB + st.slot * kSFBBytes + r * (kKSteps * kAtomBytes),
-                        p.sfb + ((size_t)(jb0 + r) * p.sf_katoms + katom0) * kAtomBytes, sf_bytes, sb);
+            tma_load_2d<kCta>(sbase + C::kOffSFA + st.slot * kSFABytes, &tmSA, fb, sx, ablk);
+            tma_load_2d<kCta>(sbase + C::kOffSFB + st.slot * kSFBBytes, &tmSB, fb, sx, jb0);
           }
           __syncwarp();
           st.next(S);
         }
       }
-      // Drain: wait until every load this thread issued into its own shared
-      // memory has landed (the scale atoms here; the leader also sees A and W
-      // of both CTAs land on its stage barriers).
+      // Drain: the leader sees every load of both CTAs land on its stage
+      // barriers (the peer stays resident until the closing cluster barrier).
       for (int s = 0; s < S; ++s) {
         const uint32_t par = (s < st.slot) ? st.phase : (st.phase ^ 1u);
-        wait_drain(sfs_bar(s), par);
         if (leader) wait_drain(full_bar(s), par);
       }
     }
@@ -586,9 +543,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!__all_sync(0xFFFFFFFFu, wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag))) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
+        // The tile's 192 W rows start at row 0 or 64 of the first scale block:
+        // its W scales start at column 0 or 2 of the 8 copied per K step.
+        const uint32_t sfb_shift = (uint32_t)(((t % p.n_tiles) * BN) % 128) / 32u;
         for (int kt = 0; kt < p.k_stages; ++kt) {
-          const bool landed = wait_bounded(full_bar(st.slot), st.phase, abort_flag) &&
-                              wait_bounded(sff_bar(sf.slot), sf.phase, abort_flag);
+          const bool landed = wait_bounded(full_bar(st.slot), st.phase, abort_flag);
           if (!__all_sync(0xFFFFFFFFu, landed)) {
             ok = false;
             break;
@@ -604,19 +563,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t adesc = adesc0 + (uint64_t)((st.slot * kABytes) >> 4);
           const uint64_t bdesc = bdesc0 + (uint64_t)((st.slot * C::kBBytes) >> 4);
           const uint32_t sf_tmem = tmem_base + (uint32_t)(kSfCol0 + sf.slot * kSfCols);
+          const uint32_t sfa_s = sbase + C::kOffSFA + st.slot * kSFABytes;
+          const uint32_t sfb_s = sbase + C::kOffSFB + st.slot * kSFBBytes;
           if (elect_one()) {
+            // Scales into this stage's TMEM scale buffer (in every CTA of the
+            // group, from its own shared memory), in issue order ahead of the
+            // MMAs that read them.
+#pragma unroll
+            for (int k = 0; k < kKSteps; ++k) {
+              tc_cp_atom<kCta>(sf_tmem + 4 * k, smem_desc(sfa_s + k * kAtomBytes, false));
+              tc_cp_atom<kCta>(sf_tmem + 4 * kKSteps + 8 * k, smem_desc(sfb_s + k * kAtomBytes, false));
+              tc_cp_atom<kCta>(sf_tmem + 4 * kKSteps + 8 * k + 4,
+                               smem_desc(sfb_s + (kKSteps + k) * kAtomBytes, false));
+            }
             if (ks == kKSteps) {
 #pragma unroll
               for (int k = 0; k < kKSteps; ++k)
                 tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
-                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
+                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
             } else {
               for (int k = 0; k < ks; ++k)
                 tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
-                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 6 * k);
+                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
             }
             tc_commit<kCta>(empty_bar(st.slot));  // the stage's shared memory (both CTAs), once read
-            tc_commit<kCta>(sfe_bar(sf.slot));    // the scale buffers (both CTAs), likewise
           }
           __syncwarp();
           st.next(S);
@@ -639,63 +609,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       wait_drain(drain_bar, 0);
-    }
-  } else if (warp >= kFirstSfWarp) {
-    // ===================== scale stagers (every CTA) =====================
-    // Lane l of the warp for quadrant q writes TMEM lane 32q + l.  A scale atom
-    // holds, at bytes 16 l .. 16 l + 15, the four K=64 scales of rows l, l+32,
-    // l+64, l+96: TMEM columns 0..3 of a K step (row r at column r/32).
-    const uint32_t lane_base = (uint32_t)(32 * (warp & 3)) << 16;
-    Ring st, sf;
-    bool ok = true;
-    for (int t = pair; t < p.num_tiles && ok; t += npairs) {
-      const bool odd = ((t % p.n_tiles) * BN) % 128 != 0;  // tile starts at row 64 of a scale block
-      for (int kt = 0; kt < p.k_stages; ++kt) {
-        if (!wait_bounded(sfs_bar(st.slot), st.phase, abort_flag) ||
-            !wait_bounded(sfe_bar(sf.slot), sf.phase ^ 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sfa_addr = sbase + C::kOffSFA + st.slot * kSFABytes + lane * 16;
-        const uint32_t sfb_addr = sbase + C::kOffSFB + st.slot * kSFBBytes + lane * 16;
-        uint32_t va[16], vb[24];
-#pragma unroll
-        for (int k = 0; k < kKSteps; ++k) {
-          const uint4 a = lds128(sfa_addr + k * kAtomBytes);
-          va[4 * k] = a.x;
-          va[4 * k + 1] = a.y;
-          va[4 * k + 2] = a.z;
-          va[4 * k + 3] = a.w;
-          const uint4 b0 = lds128(sfb_addr + k * kAtomBytes);
-          const uint4 b1 = lds128(sfb_addr + kKSteps * kAtomBytes + k * kAtomBytes);
-          // The tile's 192 rows: rows 0..191 (even tile) or 64..255 (odd tile)
-          // of the two 128-row scale blocks, 32 rows per column.
-          vb[6 * k + 0] = odd ? b0.z : b0.x;
-          vb[6 * k + 1] = odd ? b0.w : b0.y;
-          vb[6 * k + 2] = odd ? b1.x : b0.z;
-          vb[6 * k + 3] = odd ? b1.y : b0.w;
-          vb[6 * k + 4] = odd ? b1.z : b1.x;
-          vb[6 * k + 5] = odd ? b1.w : b1.y;
-        }
-        const uint32_t col = tmem_base + lane_base + (uint32_t)(kSfCol0 + sf.slot * kSfCols);
-        uint32_t v16[16], v8[8];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v16[i] = va[i];
-        tmem_st_16(col, v16);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v16[i] = vb[i];
-        tmem_st_16(col + 16, v16);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v8[i] = vb[16 + i];
-        tmem_st_8(col + 32, v8);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) arrive_leader<kCta>(leader_bar<kCta>(sff_bar(sf.slot)));
-        st.next(S);
-        sf.next(kSfBufs);
-      }
     }
   } else {
     // ===================== epilogue (every CTA) =====================
@@ -890,7 +803,8 @@ int cta_mode() {
 }
 
 template <int kCta, int kEpi>
-cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmY, const Params& p,
+cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
+                        const CUtensorMap& tmSB, const CUtensorMap& tmY, const Params& p,
                         const typename EpiSel<kEpi>::type& eq, cudaStream_t s) {
   using C = Cfg<kCta>;
   static int configured_device = -1;
@@ -935,7 +849,7 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = kCta == 2 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi>, tmA, tmB, tmY, p, eq);
+  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi>, tmA, tmB, tmSA, tmSB, tmY, p, eq);
 }
 
 }  // namespace
@@ -988,10 +902,20 @@ cudaError_t launch_linear(const uint8_t* a_codes, const uint8_t* a_scales, float
     *why = "cuTensorMapEncodeTiled failed (driver entry point missing or a layout rule violated)";
     return cudaErrorNotSupported;
   }
+  // The scale arrays (tensor-core layout) as 2-D tensors of 8-byte elements:
+  // one row per 128-row scale block (K / 64 atoms of 512 bytes), boxes of one
+  // stage's four atoms -- one block for A, the tile's two for W.
+  CUtensorMap tmSA, tmSB;
+  const uint64_t sf_row = (uint64_t)(K / kMmaK) * kAtomBytes;
+  if (!make_tensor_map_2d(&tmSA, CU_TENSOR_MAP_DATA_TYPE_UINT64, a_scales, sf_row / 8, (uint64_t)((M + 127) / 128),
+                          sf_row, kKSteps * kAtomBytes / 8, 1, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tensor_map_2d(&tmSB, CU_TENSOR_MAP_DATA_TYPE_UINT64, w_scales, sf_row / 8, (uint64_t)((N + 127) / 128),
+                          sf_row, kKSteps * kAtomBytes / 8, 2, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+    *why = "cuTensorMapEncodeTiled failed for the scale arrays";
+    return cudaErrorNotSupported;
+  }
   if (y == nullptr) tmY = tmA;  // unused by the quantizing epilogue
   Params p;
-  p.sfa = a_scales;
-  p.sfb = w_scales;
   p.bias = bias;
   p.alpha = a_g * w_g;
   p.M = (int)M;
@@ -1003,15 +927,14 @@ cudaError_t launch_linear(const uint8_t* a_codes, const uint8_t* a_scales, float
   p.num_tiles = m_tiles * p.n_tiles;
   p.k_stages = (int)((K + BK - 1) / BK);
   p.ksteps_total = (int)(K / kMmaK);
-  p.sf_katoms = (int)(K / kMmaK);
-  p.n_sfa_blocks = (int)((M + 127) / 128);
-  p.n_sfb_blocks = (int)((N + 127) / 128);
   p.stall_group = stall_group();
   if (eq == nullptr) {
     const EpiNone none;
-    return ctas == 2 ? launch_form<2, 0>(tmA, tmB, tmY, p, none, s) : launch_form<1, 0>(tmA, tmB, tmY, p, none, s);
+    return ctas == 2 ? launch_form<2, 0>(tmA, tmB, tmSA, tmSB, tmY, p, none, s)
+                     : launch_form<1, 0>(tmA, tmB, tmSA, tmSB, tmY, p, none, s);
   }
-  return ctas == 2 ? launch_form<2, 1>(tmA, tmB, tmY, p, *eq, s) : launch_form<1, 1>(tmA, tmB, tmY, p, *eq, s);
+  return ctas == 2 ? launch_form<2, 1>(tmA, tmB, tmSA, tmSB, tmY, p, *eq, s)
+                   : launch_form<1, 1>(tmA, tmB, tmSA, tmSB, tmY, p, *eq, s);
 }
 
 }  // namespace
