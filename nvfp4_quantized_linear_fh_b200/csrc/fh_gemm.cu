@@ -12,9 +12,14 @@
 // cta_group::2 (each SM computes 128 rows; the 192 W rows are split 96/96
 // between the two SMs' shared memory, so each SM loads and holds half of W);
 // the single-CTA form (128 x 192 tiles) is the same code with kCta = 1.
-// Per CTA, 192 threads:
+// Two tile forms (template parameter BN):
+//   256 (default, CTA pair): 256 x 256 output tiles, one 256-column TMEM
+//       accumulator per CTA, 4 stages, 320 threads;
+//   192 (CTA pair, or single CTA): 256 x 192 (128 x 192) tiles, two 192-column
+//       accumulators, 6 (4) stages, 192 threads.
+// Roles per CTA:
 //   warp 0      TMA producer: per 256-wide K stage, its 128 x 128-byte A tile,
-//               its (192 / kCta) x 128-byte W tile (128-byte swizzle), and the
+//               its (BN / kCta) x 128-byte W tile (128-byte swizzle), and the
 //               stage's scale atoms (512 bytes = 128 rows x 64 K; one box for
 //               this CTA's A rows, one for the tile's two W scale blocks), all
 //               by tensor TMA completing on the leader CTA's stage barrier.
@@ -23,22 +28,25 @@
 //               of two TMEM scale buffers (tcgen05.cp 32x128b.warpx4, which
 //               replicates each atom into the four lane quadrants, in both CTAs
 //               of the pair) and then issues four tcgen05.mma kind::mxf4nvf4
-//               block_scale (M = 128 kCta, N = 192, K = 64) into one of two TMEM
-//               accumulators.  Copies and MMAs run in issue order on the tensor
-//               pipe, so a scale buffer needs no barrier; double buffering
-//               keeps a copy from waiting on the MMAs still reading the other.
+//               block_scale (M = 128 kCta, N = BN, K = 64) into an accumulator.
+//               Copies and MMAs run in issue order on the tensor pipe, so a
+//               scale buffer needs no barrier; double buffering keeps a copy
+//               from waiting on the MMAs still reading the other.
 //               tcgen05.commit (multicast to the pair) frees the stage's shared
 //               memory and, after the last stage, hands the accumulator to both
 //               CTAs' epilogues.
-//   warps 2..5  epilogue: tcgen05.ld of their 32 TMEM lanes, alpha * acc + bias
-//               in FP32, BF16 round-to-nearest-even, 128-byte-swizzled staging
-//               in shared memory and TMA stores, while the MMA warp already fills
-//               the other accumulator.
-// TMEM columns (each CTA): accumulators [0, 192) and [192, 384); two scale
-// buffers of 48 columns from 384: per K=64 step, 4 columns of A scales (row r
-// at lane r%32, column r/32) then 8 columns of W scales (the two 128-row scale
-// blocks the tile's 192 rows fall in; the MMA reads 6 of them from column 0 or
-// 2).
+//   warps 2..   epilogue (4 warps for BN = 192, one per TMEM lane quadrant; 8
+//               for BN = 256, two per quadrant, one per 128-column half):
+//               tcgen05.ld of their TMEM lanes, alpha * acc + bias in FP32,
+//               BF16 round-to-nearest-even, 128-byte-swizzled staging in shared
+//               memory and TMA stores.  With two accumulators this overlaps the
+//               MMAs of the next tile; with one, each warp first copies its 128
+//               columns into registers and releases the accumulator, so the
+//               MMAs wait only for that copy.
+// TMEM columns (each CTA): the accumulators from 0, then two scale buffers of
+// 48 columns: per K=64 step, 4 columns of A scales (row r at lane r%32, column
+// r/32) then 8 columns of W scales (the two 128-row scale blocks the tile's
+// rows fall in; a 192-row tile reads 6 of them from column 0 or 2).
 // No TMA load uses cluster multicast; only tcgen05.commit is multicast.
 // Every mbarrier wait is bounded; on expiry the kernel sets the device error
 // word, stops issuing work, drains what it issued and frees its TMEM.
@@ -57,7 +65,6 @@ namespace {
 
 __device__ unsigned int g_device_error = 0;
 
-constexpr int BN = 192;                  // output columns per tile
 constexpr int BK = 256;                  // FP4 elements per stage = 128 bytes per row
 constexpr int kMmaK = 64;                // K of one tcgen05.mma kind::mxf4nvf4
 constexpr int kKSteps = BK / kMmaK;      // 4
@@ -65,22 +72,30 @@ constexpr int kAtomBytes = 512;          // 128 rows x 4 scales
 constexpr int kABytes = 128 * BK / 2;    // 16384: one CTA's 128 A rows
 constexpr int kSFABytes = kKSteps * kAtomBytes;      // 2048
 constexpr int kSFBBytes = 2 * kKSteps * kAtomBytes;  // 4096
-constexpr int kEpiWarps = 4;
 constexpr int kEpiCols = 64;                          // columns per TMA store box
 constexpr int kEpiBufBytes = 32 * kEpiCols * 2;       // 4096: 32 rows x 128 bytes
-constexpr int kThreads = 64 + 32 * kEpiWarps;         // 192
 constexpr int kTmemCols = 512;
-constexpr int kAccCols = BN;
 constexpr int kSfCols = 4 * kKSteps + 8 * kKSteps;    // 48 per stage: A 4, W 8 per K=64 step
 constexpr int kSfBufs = 2;
-constexpr int kSfCol0 = 2 * kAccCols;                 // 384
-static_assert(kSfCol0 + kSfBufs * kSfCols <= kTmemCols, "TMEM budget");
 
-template <int kCta>
+// Two tile forms share the kernel.  BN = 192: two 192-column accumulators, so
+// an epilogue overlaps the next tile's MMAs entirely; four epilogue warps.
+// BN = 256 (CTA pair only): one 256-column accumulator -- two would fill TMEM
+// -- drained into registers by eight epilogue warps (two per TMEM lane
+// quadrant, one per 128-column half), which release it before they scale,
+// round and store; each stage then feeds 33% more MACs from 12% more bytes.
+template <int kCta, int kBN>
 struct Cfg {
+  static_assert(kBN == 192 || (kBN == 256 && kCta == 2), "tile forms");
+  static constexpr int BN = kBN;                       // output columns per tile
   static constexpr int BM = 128 * kCta;                // output rows per tile
   static constexpr int kBRows = BN / kCta;             // W rows each CTA loads
-  static constexpr int kStages = kCta == 2 ? 6 : 4;
+  static constexpr int kAccBufs = BN == 256 ? 1 : 2;   // TMEM accumulators
+  static constexpr int kEpiWarps = BN == 256 ? 8 : 4;
+  static constexpr int kWarpCols = BN == 256 ? 128 : BN;  // accumulator columns per epilogue warp
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kSfCol0 = kAccBufs * BN;        // first TMEM column of the scale buffers
+  static constexpr int kStages = BN == 256 ? 4 : (kCta == 2 ? 6 : 4);
   static constexpr int kEpiBufs = kCta == 2 ? 1 : 2;   // output staging buffers per epilogue warp
   static constexpr int kBBytes = kBRows * BK / 2;
   static constexpr int kOffA = 0;
@@ -89,9 +104,9 @@ struct Cfg {
   static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
   static constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
   static constexpr int kOffBias = kOffEpi + kEpiWarps * kEpiBufs * kEpiBufBytes;
-  static constexpr int kOffBar = kOffBias + kEpiWarps * BN * 4;
-  // full, empty (per stage); acc full, acc empty (x2); drain
-  static constexpr int kNumBars = 2 * kStages + 4 + 1;
+  static constexpr int kOffBar = kOffBias + kEpiWarps * kWarpCols * 4;
+  // full, empty (per stage); acc full, acc empty (per accumulator); drain
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
   // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1
@@ -102,6 +117,7 @@ struct Cfg {
   static_assert(kOffB % 1024 == 0 && kOffSFA % 1024 == 0 && kOffEpi % 1024 == 0, "alignment");
   static_assert(kBBytes % 1024 == 0, "W stage alignment");
   static_assert(kSmemAlloc <= 232448, "shared memory budget");
+  static_assert(kSfCol0 + kSfBufs * kSfCols <= kTmemCols, "TMEM budget");
 };
 
 struct Params {
@@ -347,15 +363,15 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, bool swizzle128) {
 }
 
 template <int kCta>
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate,
-                                       uint32_t sfa_tmem, uint32_t sfb_tmem) {
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate, uint32_t sfa_tmem, uint32_t sfb_tmem) {
   if (kCta == 1) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(Cfg<1>::kIdesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
   } else {
     asm volatile(
@@ -363,7 +379,7 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X"
         " [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(Cfg<2>::kIdesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
         : "memory");
   }
 }
@@ -398,6 +414,27 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Registers written by tcgen05.ld are valid only after the wait; tying them to
+// an asm statement placed after it keeps every use of them below the wait.
+__device__ __forceinline__ void tie32(uint32_t* v) {
+  asm volatile(""
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                 "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
+                 "+r"(v[29]), "+r"(v[30]), "+r"(v[31]));
+}
+
+template <int kC>
+__device__ __forceinline__ void tmem_ld_wait_tied(uint32_t (&v)[kC][64]) {
+  tmem_ld_wait();
+#pragma unroll
+  for (int c = 0; c < kC; ++c) {
+    tie32(&v[c][0]);
+    tie32(&v[c][32]);
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -418,14 +455,15 @@ struct Ring {
   }
 };
 
-template <int kCta, int kEpi>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int kCta, int kEpi, int kBN>
+__global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
     nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                         const __grid_constant__ CUtensorMap tmY, const Params p,
                         const __grid_constant__ typename EpiSel<kEpi>::type eq) {
-  using C = Cfg<kCta>;
+  using C = Cfg<kCta, kBN>;
   constexpr int S = C::kStages;
+  constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
@@ -434,12 +472,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto full_bar = [&](int s) { return bar0 + 8u * s; };            // leader: A, W and scales landed (both CTAs)
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };     // each CTA: stage free again
   auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };  // each CTA: accumulator ready
-  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };  // leader: accumulator drained
-  const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + C::kAccBufs + a); };  // leader: accumulator drained
+  const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * C::kAccBufs);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kNumBars * 8);
   if constexpr (kEpi == 1) {
     // The next layer's decision table, in the (otherwise unused) output staging area.
-    static_assert(sizeof(QuantTable) <= kEpiWarps * C::kEpiBufs * kEpiBufBytes, "table fits the staging area");
+    static_assert(sizeof(QuantTable) <= C::kEpiWarps * C::kEpiBufs * kEpiBufBytes, "table fits the staging area");
     const uint4* src = reinterpret_cast<const uint4*>(&eq.tab);
     uint4* dst = reinterpret_cast<uint4*>(smem + C::kOffEpi);
     for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 16); i += blockDim.x) dst[i] = src[i];
@@ -458,9 +496,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(full_bar(s), kCta);
       mbar_init(empty_bar(s), 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < C::kAccBufs; ++a) {
       mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), kEpiWarps * kCta);
+      mbar_init(acce_bar(a), C::kEpiWarps * kCta);
     }
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
@@ -542,9 +580,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = pair; t < p.num_tiles && ok; t += npairs) {
         if (!__all_sync(0xFFFFFFFFu, wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag))) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kAccCols);
-        // The tile's 192 W rows start at row 0 or 64 of the first scale block:
-        // its W scales start at column 0 or 2 of the 8 copied per K step.
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        // A 192-row W tile starts at row 0 or 64 of its first scale block: its
+        // W scales start at column 0 or 2 of the 8 copied per K step (a
+        // 256-row tile always at 0).
         const uint32_t sfb_shift = (uint32_t)(((t % p.n_tiles) * BN) % 128) / 32u;
         for (int kt = 0; kt < p.k_stages; ++kt) {
           const bool landed = wait_bounded(full_bar(st.slot), st.phase, abort_flag);
@@ -562,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int ks = min(kKSteps, p.ksteps_total - kt * kKSteps);
           const uint64_t adesc = adesc0 + (uint64_t)((st.slot * kABytes) >> 4);
           const uint64_t bdesc = bdesc0 + (uint64_t)((st.slot * C::kBBytes) >> 4);
-          const uint32_t sf_tmem = tmem_base + (uint32_t)(kSfCol0 + sf.slot * kSfCols);
+          const uint32_t sf_tmem = tmem_base + (uint32_t)(C::kSfCol0 + sf.slot * kSfCols);
           const uint32_t sfa_s = sbase + C::kOffSFA + st.slot * kSFABytes;
           const uint32_t sfb_s = sbase + C::kOffSFB + st.slot * kSFBBytes;
           if (elect_one()) {
@@ -580,11 +619,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int k = 0; k < kKSteps; ++k)
                 tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
-                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
+                             C::kIdesc, (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
             } else {
               for (int k = 0; k < ks; ++k)
                 tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
-                             (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
+                             C::kIdesc, (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
             }
             tc_commit<kCta>(empty_bar(st.slot));  // the stage's shared memory (both CTAs), once read
           }
@@ -595,7 +634,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (elect_one()) tc_commit<kCta>(accf_bar(acc));  // accumulator ready for both CTAs' epilogues
         __syncwarp();
-        if (++acc == 2) {
+        if (++acc == C::kAccBufs) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -612,10 +651,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ===================== epilogue (every CTA) =====================
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // Warp ew = warp - 2 reads TMEM lane quadrant warp % 4 (32 output rows)
+    // and accumulator columns [hcol, hcol + kWarpCols).
+    constexpr int kWarpCols = C::kWarpCols;
+    constexpr int kChunks = kWarpCols / kEpiCols;
+    const int ew = warp - 2;
+    const int q = warp & 3;
+    const int hcol = (ew >> 2) * kWarpCols;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    uint8_t* stage_buf = smem + C::kOffEpi + (warp - 2) * C::kEpiBufs * kEpiBufBytes;
-    float* bias_s = reinterpret_cast<float*>(smem + C::kOffBias) + (warp - 2) * BN;
+    uint8_t* stage_buf = smem + C::kOffEpi + ew * C::kEpiBufs * kEpiBufBytes;
+    float* bias_s = reinterpret_cast<float*>(smem + C::kOffBias) + ew * kWarpCols;
     int acc = 0;
     uint32_t acc_phase = 0;
     int buf = 0;
@@ -623,10 +668,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = pair; t < p.num_tiles; t += npairs) {
       const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
       const int row0 = m_tile * C::BM + (int)rank * 128 + 32 * q;  // this warp's 32 output rows
-      const int n0 = n_tile * BN;
-      // The tile's bias, in FP32, staged in this warp's shared memory before
-      // the accumulator is ready (lanes 0..23 load 8 values each).
-      if (lane < BN / 8) {
+      const int n0 = n_tile * BN + hcol;                           // this warp's first column
+      // The warp's bias columns in FP32, staged in its shared memory before the
+      // accumulator is ready (8 values per lane).
+      if (lane < kWarpCols / 8) {
         uint4 u = make_uint4(0, 0, 0, 0);
         if (p.bias != nullptr && n0 + 8 * lane < p.N)
           u = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * lane));
@@ -641,23 +686,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (!wait_bounded(accf_bar(acc), acc_phase, abort_flag)) break;
       tc_fence_after();
-      for (int c = 0; c < BN / kEpiCols; ++c) {
+      const uint32_t tcol = tmem_base + lane_base + (uint32_t)(acc * BN + hcol);
+      // One 64-column chunk from raw accumulator bits: y = alpha * acc + bias,
+      // BF16, then either the quantizing epilogue or a TMA store of y.
+      auto emit = [&](const uint32_t(&v)[64], int c) {
         const int col0 = n0 + c * kEpiCols;
-        if (col0 >= p.N) break;  // warp-uniform
-        uint32_t v[2][32];
-        const uint32_t taddr = tmem_base + lane_base + (uint32_t)(acc * kAccCols + c * kEpiCols);
-        tmem_ld_32(taddr, v[0]);
-        tmem_ld_32(taddr + 32, v[1]);
-        tmem_ld_wait();
         uint32_t packed[32];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const float4 bv = reinterpret_cast<const float4*>(bias_s + c * kEpiCols)[j];
-          const int cc = 4 * j;
-          const float y0 = fmaf(p.alpha, __uint_as_float(v[cc >> 5][cc & 31]), bv.x);
-          const float y1 = fmaf(p.alpha, __uint_as_float(v[(cc + 1) >> 5][(cc + 1) & 31]), bv.y);
-          const float y2 = fmaf(p.alpha, __uint_as_float(v[(cc + 2) >> 5][(cc + 2) & 31]), bv.z);
-          const float y3 = fmaf(p.alpha, __uint_as_float(v[(cc + 3) >> 5][(cc + 3) & 31]), bv.w);
+          const float y0 = fmaf(p.alpha, __uint_as_float(v[4 * j]), bv.x);
+          const float y1 = fmaf(p.alpha, __uint_as_float(v[4 * j + 1]), bv.y);
+          const float y2 = fmaf(p.alpha, __uint_as_float(v[4 * j + 2]), bv.z);
+          const float y3 = fmaf(p.alpha, __uint_as_float(v[4 * j + 3]), bv.w);
           packed[2 * j] = pack_bf16x2(y0, y1);
           packed[2 * j + 1] = pack_bf16x2(y2, y3);
         }
@@ -686,35 +727,60 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (row < eq.m_pad)
             *reinterpret_cast<uint32_t*>(eq.scales + ((size_t)(row >> 7) * eq.katoms + (col0 >> 6)) * 512 +
                                          (row & 31) * 16 + ((row >> 5) & 3) * 4) = row < p.M ? word : 0u;
-          continue;
-        }
-        // Reuse a staging buffer only after its previous TMA store has read it.
-        if (lane == 0) {
-          if (C::kEpiBufs == 1)
-            bulk_wait_read_0();
-          else
-            bulk_wait_read_1();
-        }
-        __syncwarp();
-        uint8_t* sb = stage_buf + buf * kEpiBufBytes;
-        const uint32_t row = (uint32_t)lane;
+        } else {
+          // Reuse a staging buffer only after its previous TMA store has read it.
+          if (lane == 0) {
+            if (C::kEpiBufs == 1)
+              bulk_wait_read_0();
+            else
+              bulk_wait_read_1();
+          }
+          __syncwarp();
+          uint8_t* sb = stage_buf + buf * kEpiBufBytes;
+          const uint32_t row = (uint32_t)lane;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t chunk = (uint32_t)i ^ (row & 7u);  // 128-byte swizzle
-          *reinterpret_cast<uint4*>(sb + row * 128 + chunk * 16) =
-              make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          for (int i = 0; i < 8; ++i) {
+            const uint32_t chunk = (uint32_t)i ^ (row & 7u);  // 128-byte swizzle
+            *reinterpret_cast<uint4*>(sb + row * 128 + chunk * 16) =
+                make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.M) tma_store_2d(&tmY, smem_u32(sb), col0, row0);  // rows past M: nothing to store
+          if (lane == 0) bulk_commit();
+          if (C::kEpiBufs == 2) buf ^= 1;
         }
-        fence_proxy_async_smem();
+      };
+      auto release = [&]() {  // all TMEM reads of this accumulator are done: hand it back
+        tc_fence_before();
         __syncwarp();
-        if (lane == 0 && row0 < p.M) tma_store_2d(&tmY, smem_u32(sb), col0, row0);  // rows past M: nothing to store
-        if (lane == 0) bulk_commit();
-        if (C::kEpiBufs == 2) buf ^= 1;
+        if (lane == 0) arrive_leader<kCta>(leader_bar<kCta>(acce_bar(acc)));
+      };
+      if constexpr (C::kAccBufs == 1) {
+        // One accumulator: copy this warp's columns out, release, then emit.
+        uint32_t v[kChunks][64];
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          tmem_ld_32(tcol + c * kEpiCols, *reinterpret_cast<uint32_t(*)[32]>(&v[c][0]));
+          tmem_ld_32(tcol + c * kEpiCols + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c][32]));
+        }
+        tmem_ld_wait_tied(v);
+        release();
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c)
+          if (n0 + c * kEpiCols < p.N) emit(v[c], c);  // warp-uniform
+      } else {
+        for (int c = 0; c < kChunks; ++c) {
+          if (n0 + c * kEpiCols >= p.N) break;  // warp-uniform
+          uint32_t v[64];
+          tmem_ld_32(tcol + c * kEpiCols, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+          tmem_ld_32(tcol + c * kEpiCols + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+          tmem_ld_wait();
+          emit(v, c);
+        }
+        release();
       }
-      // All TMEM reads of this accumulator are done: hand it back to the MMA warp.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) arrive_leader<kCta>(leader_bar<kCta>(acce_bar(acc)));
-      if (++acc == 2) {
+      if (++acc == C::kAccBufs) {
         acc = 0;
         acc_phase ^= 1u;
       }
@@ -802,18 +868,31 @@ int cta_mode() {
   return mode;
 }
 
-template <int kCta, int kEpi>
+// Tile width of the CTA-pair form for an N-column output: 256 unless the
+// environment variable FH_GEMM_BN (read at first launch) is 192.
+int tile_width(int64_t N) {
+  static int forced = -1;
+  if (forced < 0) {
+    const char* e = getenv("FH_GEMM_BN");
+    forced = (e != nullptr && strcmp(e, "192") == 0) ? 192 : (e != nullptr && strcmp(e, "256") == 0) ? 256 : 0;
+  }
+  if (forced != 0) return forced;
+  (void)N;
+  return 256;
+}
+
+template <int kCta, int kEpi, int kBN>
 cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
                         const CUtensorMap& tmSB, const CUtensorMap& tmY, const Params& p,
                         const typename EpiSel<kEpi>::type& eq, cudaStream_t s) {
-  using C = Cfg<kCta>;
+  using C = Cfg<kCta, kBN>;
   static int configured_device = -1;
   static int max_groups = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
     cudaError_t e =
-        cudaFuncSetAttribute(nvfp4_linear_kernel<kCta, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+        cudaFuncSetAttribute(nvfp4_linear_kernel<kCta, kEpi, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
     if (e != cudaSuccess) return e;
     max_groups = sm_count() / kCta;
     if (kCta == 2) {
@@ -825,12 +904,13 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
       attr[0].val.clusterDim.y = 1;
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(2 * max_groups);
-      cfg.blockDim = dim3(kThreads);
+      cfg.blockDim = dim3(C::kThreads);
       cfg.dynamicSmemBytes = C::kSmemAlloc;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4_linear_kernel<2, kEpi>, &cfg) == cudaSuccess && clusters > 0)
+      if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4_linear_kernel<2, kEpi, kBN>, &cfg) == cudaSuccess &&
+          clusters > 0)
         max_groups = clusters < max_groups ? clusters : max_groups;
       cudaGetLastError();
     }
@@ -844,12 +924,12 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(groups * kCta);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemAlloc;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = kCta == 2 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi>, tmA, tmB, tmSA, tmSB, tmY, p, eq);
+  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi, kBN>, tmA, tmB, tmSA, tmSB, tmY, p, eq);
 }
 
 }  // namespace
@@ -891,6 +971,7 @@ cudaError_t launch_linear(const uint8_t* a_codes, const uint8_t* a_scales, float
                           const uint8_t* w_scales, float w_g, const uint16_t* bias, uint16_t* y, int64_t M,
                           int64_t N, int64_t K, const EpiQuant* eq, cudaStream_t s, const char** why) {
   const int ctas = cta_mode();
+  const int BN = ctas == 2 ? tile_width(N) : 192;
   CUtensorMap tmA, tmB, tmY;
   const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
   if (!make_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M,
@@ -930,11 +1011,13 @@ cudaError_t launch_linear(const uint8_t* a_codes, const uint8_t* a_scales, float
   p.stall_group = stall_group();
   if (eq == nullptr) {
     const EpiNone none;
-    return ctas == 2 ? launch_form<2, 0>(tmA, tmB, tmSA, tmSB, tmY, p, none, s)
-                     : launch_form<1, 0>(tmA, tmB, tmSA, tmSB, tmY, p, none, s);
+    if (ctas == 1) return launch_form<1, 0, 192>(tmA, tmB, tmSA, tmSB, tmY, p, none, s);
+    return BN == 256 ? launch_form<2, 0, 256>(tmA, tmB, tmSA, tmSB, tmY, p, none, s)
+                     : launch_form<2, 0, 192>(tmA, tmB, tmSA, tmSB, tmY, p, none, s);
   }
-  return ctas == 2 ? launch_form<2, 1>(tmA, tmB, tmSA, tmSB, tmY, p, *eq, s)
-                   : launch_form<1, 1>(tmA, tmB, tmSA, tmSB, tmY, p, *eq, s);
+  if (ctas == 1) return launch_form<1, 1, 192>(tmA, tmB, tmSA, tmSB, tmY, p, *eq, s);
+  return BN == 256 ? launch_form<2, 1, 256>(tmA, tmB, tmSA, tmSB, tmY, p, *eq, s)
+                   : launch_form<2, 1, 192>(tmA, tmB, tmSA, tmSB, tmY, p, *eq, s);
 }
 
 }  // namespace
