@@ -142,7 +142,9 @@ int fh_gelu_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ld
  * (see fh_device_status) instead of hanging; the kernel then drains the
  * copies and MMAs it issued and frees its TMEM before it exits.
  * Environment: FH_GEMM_CTAS=1 (read at the first launch) selects the
- * single-CTA form (128-row tiles) instead of the CTA pair;
+ * single-CTA form (128-row tiles) instead of the CTA pair; FH_GEMM_BN=192
+ * (read at the first launch) makes the CTA pair use 256 x 192 tiles instead
+ * of the default 256 x 256 (both give identical results);
  * FH_GEMM_TEST_STALL=1 (read at each launch) is a test hook that makes the
  * first CTA group's MMA warp stop after three stages of its first tile
  * (K >= 1024), so the call ends with FH_ERR_TIMEOUT. */
