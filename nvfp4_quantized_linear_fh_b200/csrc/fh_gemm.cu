@@ -14,7 +14,7 @@
 // the single-CTA form (128 x 192 tiles) is the same code with kCta = 1.
 // Two tile forms (template parameter BN):
 //   256 (default, CTA pair): 256 x 256 output tiles, one 256-column TMEM
-//       accumulator per CTA, 4 stages, 320 threads;
+//       accumulator per CTA, 5 stages, 320 threads;
 //   192 (CTA pair, or single CTA): 256 x 192 (128 x 192) tiles, two 192-column
 //       accumulators, 6 (4) stages, 192 threads.
 // Roles per CTA:
@@ -95,7 +95,7 @@ struct Cfg {
   static constexpr int kWarpCols = BN == 256 ? 128 : BN;  // accumulator columns per epilogue warp
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kSfCol0 = kAccBufs * BN;        // first TMEM column of the scale buffers
-  static constexpr int kStages = BN == 256 ? 4 : (kCta == 2 ? 6 : 4);
+  static constexpr int kStages = BN == 256 ? 5 : (kCta == 2 ? 6 : 4);
   static constexpr int kEpiBufs = kCta == 2 ? 1 : 2;   // output staging buffers per epilogue warp
   static constexpr int kBBytes = kBRows * BK / 2;
   static constexpr int kOffA = 0;
@@ -104,7 +104,7 @@ struct Cfg {
   static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
   static constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
   static constexpr int kOffBias = kOffEpi + kEpiWarps * kEpiBufs * kEpiBufBytes;
-  static constexpr int kOffBar = kOffBias + kEpiWarps * kWarpCols * 4;
+  static constexpr int kOffBar = kOffBias + kEpiWarps * kWarpCols * 2;
   // full, empty (per stage); acc full, acc empty (per accumulator); drain
   static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
     const int hcol = (ew >> 2) * kWarpCols;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     uint8_t* stage_buf = smem + C::kOffEpi + ew * C::kEpiBufs * kEpiBufBytes;
-    float* bias_s = reinterpret_cast<float*>(smem + C::kOffBias) + ew * kWarpCols;
+    uint32_t* bias_s = reinterpret_cast<uint32_t*>(smem + C::kOffBias) + ew * (kWarpCols / 2);  // BF16 pairs
     int acc = 0;
     uint32_t acc_phase = 0;
     int buf = 0;
@@ -669,19 +669,13 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
       const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
       const int row0 = m_tile * C::BM + (int)rank * 128 + 32 * q;  // this warp's 32 output rows
       const int n0 = n_tile * BN + hcol;                           // this warp's first column
-      // The warp's bias columns in FP32, staged in its shared memory before the
-      // accumulator is ready (8 values per lane).
+      // The warp's bias columns (BF16 pairs), staged in its shared memory
+      // before the accumulator is ready (8 values per lane).
       if (lane < kWarpCols / 8) {
         uint4 u = make_uint4(0, 0, 0, 0);
         if (p.bias != nullptr && n0 + 8 * lane < p.N)
           u = __ldg(reinterpret_cast<const uint4*>(p.bias + n0 + 8 * lane));
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-        float4 f0 = make_float4(__uint_as_float(w[0] << 16), __uint_as_float(w[0] & 0xFFFF0000u),
-                                __uint_as_float(w[1] << 16), __uint_as_float(w[1] & 0xFFFF0000u));
-        float4 f1 = make_float4(__uint_as_float(w[2] << 16), __uint_as_float(w[2] & 0xFFFF0000u),
-                                __uint_as_float(w[3] << 16), __uint_as_float(w[3] & 0xFFFF0000u));
-        reinterpret_cast<float4*>(bias_s)[2 * lane] = f0;
-        reinterpret_cast<float4*>(bias_s)[2 * lane + 1] = f1;
+        reinterpret_cast<uint4*>(bias_s)[lane] = u;
       }
       __syncwarp();
       if (!wait_bounded(accf_bar(acc), acc_phase, abort_flag)) break;
@@ -694,11 +688,11 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
         uint32_t packed[32];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float4 bv = reinterpret_cast<const float4*>(bias_s + c * kEpiCols)[j];
-          const float y0 = fmaf(p.alpha, __uint_as_float(v[4 * j]), bv.x);
-          const float y1 = fmaf(p.alpha, __uint_as_float(v[4 * j + 1]), bv.y);
-          const float y2 = fmaf(p.alpha, __uint_as_float(v[4 * j + 2]), bv.z);
-          const float y3 = fmaf(p.alpha, __uint_as_float(v[4 * j + 3]), bv.w);
+          const uint2 bw = reinterpret_cast<const uint2*>(bias_s + c * (kEpiCols / 2))[j];
+          const float y0 = fmaf(p.alpha, __uint_as_float(v[4 * j]), __uint_as_float(bw.x << 16));
+          const float y1 = fmaf(p.alpha, __uint_as_float(v[4 * j + 1]), __uint_as_float(bw.x & 0xFFFF0000u));
+          const float y2 = fmaf(p.alpha, __uint_as_float(v[4 * j + 2]), __uint_as_float(bw.y << 16));
+          const float y3 = fmaf(p.alpha, __uint_as_float(v[4 * j + 3]), __uint_as_float(bw.y & 0xFFFF0000u));
           packed[2 * j] = pack_bf16x2(y0, y1);
           packed[2 * j + 1] = pack_bf16x2(y2, y3);
         }
