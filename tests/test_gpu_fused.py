@@ -134,6 +134,18 @@ def test_fused_single_cta_form():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
 
 
+def test_fused_192_wide_pair_form():
+    """The 256 x 192-tile CTA-pair form (FH_GEMM_BN=192) with the fused epilogue."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, FH_GEMM_BN="192")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", os.path.abspath(__file__),
+                        "-k", "matches_three_calls or clip_counts"],
+                       env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
 @pytest.mark.parametrize("M,K", [(100, 192), (129, 512), (300, 2688), (1, 64), (513, 10752)])
 def test_gelu_quantize_matches_two_calls(M, K):
     """fh_gelu_quantize_act == fh_gelu_bf16 then fh_quantize_act, bit for bit

@@ -153,6 +153,66 @@ def test_single_cta_form_matches_oracle():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
 
 
+def test_192_wide_pair_form_matches_oracle():
+    """The 256 x 192-tile CTA-pair form (FH_GEMM_BN=192: two accumulators, four
+    epilogue warps) passes the same parity cases as the default 256-wide form."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, FH_GEMM_BN="192")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "gpu", os.path.abspath(__file__),
+                        "-k", "small or tiny or no_bias or back_to_back or full_size"],
+                       env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+_FORM_HASH = r"""
+import hashlib, sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import nvfp4_quantized_linear_fh_b200 as fh
+import synthetic as S
+out = []
+for (M, K, N) in [(700, 2688, 8064), (333, 1024, 200), (4100, 10752, 2688)]:
+    def dev(b):
+        return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).cuda().view(torch.bfloat16)
+    x = dev(S.random_bf16(("forms", M, "x"), (M, K), 1.0))
+    w = dev(S.random_bf16(("forms", M, "w"), (N, K), 0.02))
+    b = dev(S.random_bf16(("forms", M, "b"), (N,), 0.1))
+    ac, asc = fh.empty_quantized(M, K); wc, wsc = fh.empty_quantized(N, K)
+    fh.fh_quantize_act(x, 1.0 / 256, ac, asc, None); fh.fh_quantize_act(w, 1.0 / 8192, wc, wsc, None)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    fh.fh_nvfp4_linear(ac, asc, 1.0 / 256, wc, wsc, 1.0 / 8192, b, y)
+    g, gs = fh.empty_quantized(M, N) if N % 64 == 0 else (None, None)
+    if g is not None:
+        fh.fh_nvfp4_linear_gelu_quant(ac, asc, 1.0 / 256, wc, wsc, 1.0 / 8192, b, 1.0 / 512, g, gs, None)
+    torch.cuda.synchronize()
+    h = hashlib.sha256(y.view(torch.int16).cpu().numpy().tobytes())
+    if g is not None:
+        h.update(g.cpu().numpy().tobytes()); h.update(gs.cpu().numpy().tobytes())
+    out.append(h.hexdigest()[:16])
+fh.fh_device_status()
+print(" ".join(out))
+"""
+
+
+def test_kernel_forms_are_bit_identical():
+    """The 256-wide pair form (default), the 192-wide pair form and the
+    single-CTA form accumulate in the same order: y, and the fused epilogue's
+    codes and scales, are byte-identical across them (ragged M, N and K)."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    hashes = {}
+    for name, extra in (("256 pair", {}), ("192 pair", {"FH_GEMM_BN": "192"}), ("single CTA", {"FH_GEMM_CTAS": "1"})):
+        env = dict(os.environ, **extra)
+        r = subprocess.run([sys.executable, "-c", _FORM_HASH, root], env=env, capture_output=True, text=True,
+                           timeout=600)
+        assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-2000:]
+        hashes[name] = r.stdout.strip().splitlines()[-1]
+    assert len(set(hashes.values())) == 1, hashes
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     """A wait that nothing satisfies gives up after its limit, the host reads
     FH_ERR_TIMEOUT, and the next GEMM still runs correctly."""
@@ -173,7 +233,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
 def test_gemm_stall_times_out_drains_and_context_survives(monkeypatch):
     """With the test hook FH_GEMM_TEST_STALL=1 the first CTA pair's MMA warp
     stops issuing after three stages of its first tile, without committing.
-    That pair's producer, scale stagers and epilogue then run into their
+    That pair's producer and epilogue then run into their
     bounded waits (about 4 s) while copies and MMAs are in flight; the kernel
     drains them and frees TMEM, and the host reads FH_ERR_TIMEOUT.  With the
     hook off, the next GEMM in the same context passes parity."""
