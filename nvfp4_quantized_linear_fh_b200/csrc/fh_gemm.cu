@@ -525,6 +525,10 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
   if (kCta == 2) cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent of the preceding kernel (typically the
+  // quantizer that wrote A): the setup above overlapped its tail; nothing below
+  // touches global memory before that kernel has completed.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ===================== TMA producer (every CTA) =====================
@@ -912,17 +916,22 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
   }
   const int groups = p.num_tiles < max_groups ? p.num_tiles : max_groups;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kCta;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int nattr = 0;
+  attr[nattr].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[nattr++].val.programmaticStreamSerializationAllowed = 1;
+  if (kCta == 2) {
+    attr[nattr].id = cudaLaunchAttributeClusterDimension;
+    attr[nattr].val.clusterDim.x = kCta;
+    attr[nattr].val.clusterDim.y = 1;
+    attr[nattr++].val.clusterDim.z = 1;
+  }
   cfg.gridDim = dim3(groups * kCta);
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemAlloc;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = kCta == 2 ? 1 : 0;
+  cfg.numAttrs = nattr;
   return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi, kBN>, tmA, tmB, tmSA, tmSB, tmY, p, eq);
 }
 

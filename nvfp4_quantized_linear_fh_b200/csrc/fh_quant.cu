@@ -453,6 +453,10 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmx)) : "memory");
   }
   __syncthreads();
+  // A kernel launched as this one's programmatic dependent (the GEMM that
+  // reads its output) may start its setup now; it waits for this grid to
+  // complete before it reads anything.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nb = p.K >> 4;
