@@ -176,6 +176,32 @@ int fh_nvfp4_linear_gelu_quant(const uint8_t* a_codes_dev, const uint8_t* a_scal
                                uint8_t* out_scales_dev, unsigned long long* out_clip_count_dev,
                                int64_t M, int64_t N, int64_t K, fh_stream_t stream);
 
+/* The layer on host buffers: y_host = bf16(a_g * w_g * Q(x_host) . W^T + bias),
+ * quantizing x with a_gscale exactly as fh_quantize_act and multiplying as
+ * fh_nvfp4_linear, so y_host is byte-identical to those two calls on the same
+ * rows.  x_host: BF16 [M, K] in host memory; y_host: BF16 [M, N] in host memory,
+ * written; both should be page-locked (cudaHostAlloc / cudaHostRegister) --
+ * pageable memory works, but then the copies do not overlap.  Weights, bias and
+ * the clip counter (may be NULL) are device memory as in fh_nvfp4_linear.
+ * The rows are processed in chunks of chunk_rows (a multiple of 128): each
+ * chunk's upload, quantization and GEMM run on `stream` while the previous
+ * chunk's download runs on a copy stream the library keeps per host thread and
+ * device, so transfers in both directions and the kernels overlap.  The call
+ * is ordered on `stream` like any other: work enqueued there afterwards sees
+ * y_host complete (synchronize before reading it on the host).
+ * workspace_dev: device memory owned by the caller, 256-byte aligned, at least
+ * fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows) bytes (two x chunks,
+ * the chunk's codes and scales, two y chunks); the library allocates none.
+ * Shape rules as fh_nvfp4_linear (K % 64 == 0, N % 8 == 0). */
+int fh_nvfp4_linear_host(const uint16_t* x_host, int64_t M, int64_t K, float a_gscale, const uint8_t* w_codes_dev,
+                         const uint8_t* w_scales_dev, float w_gscale, const uint16_t* bias_dev, int64_t N,
+                         uint16_t* y_host, unsigned long long* clip_count_dev, int64_t chunk_rows,
+                         void* workspace_dev, size_t workspace_bytes, fh_stream_t stream);
+
+/* Workspace bytes fh_nvfp4_linear_host needs for K, N and chunk_rows; 0 if the
+ * shape is not supported. */
+size_t fh_nvfp4_linear_host_workspace_bytes(int64_t K, int64_t N, int64_t chunk_rows);
+
 /* Permute FH_SCALES_MMA_TILED scales of a [rows, K] matrix into row-major
  * [rows, K/16] (drops the padding).  Requires K % 64 == 0. */
 int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows,

@@ -59,6 +59,9 @@ _SIG = {
     "fh_nvfp4_linear_gelu_quant": (_c.c_int, [_P, _P, _c.c_float, _P, _P, _c.c_float, _P, _c.c_float, _P, _P, _P,
                                               _I64, _I64, _I64, _P]),
     "fh_scales_to_rowmajor": (_c.c_int, [_P, _P, _I64, _I64, _P]),
+    "fh_nvfp4_linear_host": (_c.c_int, [_P, _I64, _I64, _c.c_float, _P, _P, _c.c_float, _P, _I64, _P, _P, _I64, _P,
+                                        _c.c_size_t, _P]),
+    "fh_nvfp4_linear_host_workspace_bytes": (_c.c_size_t, [_I64, _I64, _I64]),
     "fh_gelu_bf16": (_c.c_int, [_P, _P, _I64, _P]),
     "fh_quantize_int8_rows": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fh_int8_attention_scores": (_c.c_int, [_P, _P, _P, _P, _c.c_float, _P, _I64, _I64, _I64, _I64, _P]),
@@ -229,6 +232,42 @@ def fh_nvfp4_linear_gelu_quant(a_codes: torch.Tensor, a_scales: torch.Tensor, a_
                                            _ptr(w_scales), float(w_gscale), _ptr(bias), float(out_gscale),
                                            _ptr(out_codes), _ptr(out_scales), _ptr(out_clip), M, N, K,
                                            _stream(stream)))
+
+
+def fh_nvfp4_linear_host_workspace_bytes(K: int, N: int, chunk_rows: int = 4096) -> int:
+    return _lib.fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows)
+
+
+def fh_nvfp4_linear_host(x_host: torch.Tensor, a_gscale: float, w_codes: torch.Tensor, w_scales: torch.Tensor,
+                         w_gscale: float, bias: torch.Tensor | None, y_host: torch.Tensor,
+                         clip: torch.Tensor | None = None, chunk_rows: int = 4096,
+                         workspace: torch.Tensor | None = None, stream=None) -> None:
+    """y_host [M, N] = the NVFP4 layer on x_host [M, K]: host BF16 tensors (pin them for overlap), weights on the
+    device; chunked upload, quantize, GEMM and download overlap (see include/fh.h).  Ordered on the stream:
+    synchronize before reading y_host.  workspace: CUDA uint8 of fh_nvfp4_linear_host_workspace_bytes bytes, or
+    None to allocate one for this call."""
+    for t, n in ((x_host, "x_host"), (y_host, "y_host")):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or t.dtype not in _BF16 or t.dim() != 2:
+            raise TypeError(f"{n} must be a 2-D BF16 CPU tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(w_codes, _U8, "w_codes", 2)
+    _need(w_scales, _U8, "w_scales")
+    M, K = x_host.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K or tuple(y_host.shape) != (M, N):
+        raise ValueError("shape mismatch: x_host [M, K], w_codes [N, K/2], y_host [M, N]")
+    if bias is not None:
+        _need(bias, _BF16, "bias")
+    if clip is not None and (clip.dtype != torch.int64 or clip.device.type != "cuda"):
+        raise TypeError("clip must be a CUDA int64 tensor")
+    need = fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=w_codes.device)
+    _need(workspace, _U8, "workspace")
+    _check(_lib.fh_nvfp4_linear_host(_P(x_host.data_ptr()), M, K, float(a_gscale), _ptr(w_codes), _ptr(w_scales),
+                                     float(w_gscale), _ptr(bias), N, _P(y_host.data_ptr()), _ptr(clip), chunk_rows,
+                                     _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def fh_scales_to_rowmajor(tiled: torch.Tensor, rowmajor: torch.Tensor, rows: int, K: int, stream=None) -> None:

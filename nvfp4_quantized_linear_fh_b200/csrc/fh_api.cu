@@ -208,6 +208,48 @@ int fh_nvfp4_linear_gelu_quant(const uint8_t* a_codes_dev, const uint8_t* a_scal
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear_gelu_quant launch");
 }
 
+size_t fh_nvfp4_linear_host_workspace_bytes(int64_t K, int64_t N, int64_t chunk_rows) {
+  if (K <= 0 || K % 64 != 0 || N <= 0 || N % 8 != 0 || chunk_rows <= 0 || chunk_rows % 128 != 0 ||
+      K > 0x7FFFFFFF || N > 0x7FFFFFFF || chunk_rows > 0x7FFFFFFF)
+    return 0;
+  return fh::host_linear_workspace_bytes(K, N, chunk_rows);
+}
+
+int fh_nvfp4_linear_host(const uint16_t* x_host, int64_t M, int64_t K, float a_gscale, const uint8_t* w_codes_dev,
+                         const uint8_t* w_scales_dev, float w_gscale, const uint16_t* bias_dev, int64_t N,
+                         uint16_t* y_host, unsigned long long* clip_count_dev, int64_t chunk_rows,
+                         void* workspace_dev, size_t workspace_bytes, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!(a_gscale > 0.0f) || isinf(a_gscale) || !(w_gscale > 0.0f) || isinf(w_gscale))
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_host: global scales must be finite and > 0%s");
+  if (M < 0 || M > 0x7FFFFFFF)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_host: need 0 <= M < 2^31%s");
+  const size_t need = fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows);
+  if (need == 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_nvfp4_linear_host: need K > 0, K %% 64 == 0, N > 0, N %% 8 == 0, chunk_rows > 0, "
+                "chunk_rows %% 128 == 0%s");
+  if (M == 0) return FH_OK;
+  if (x_host == nullptr || y_host == nullptr || w_codes_dev == nullptr || w_scales_dev == nullptr ||
+      workspace_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_host: null pointer%s");
+  if (workspace_bytes < need)
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_host: workspace smaller than "
+                                    "fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows)%s");
+  if ((reinterpret_cast<uintptr_t>(workspace_dev) & 255u) != 0 || !aligned16(w_codes_dev) ||
+      !aligned16(w_scales_dev) || (bias_dev != nullptr && !aligned16(bias_dev)))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_nvfp4_linear_host: workspace must be 256-byte aligned, weights and bias 16-byte aligned%s");
+  if (int st = check_device()) return st;
+  const char* why = nullptr;
+  cudaError_t e = fh::launch_nvfp4_linear_host(x_host, M, K, a_gscale, w_codes_dev, w_scales_dev, w_gscale, bias_dev,
+                                               N, y_host, clip_count_dev, chunk_rows, workspace_dev,
+                                               (cudaStream_t)stream, &why);
+  if (e == cudaErrorNotSupported && why != nullptr)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_host: %s", why);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear_host");
+}
+
 int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows, int64_t K,
                           fh_stream_t stream) {
   g_last_error[0] = 0;

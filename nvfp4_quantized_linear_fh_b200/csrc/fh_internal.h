@@ -92,4 +92,12 @@ cudaError_t launch_adaln_modulation(const uint16_t* e, int64_t bt, int64_t d, co
                                     const uint16_t* proj, const uint16_t* bias, int64_t L, int64_t n, float* code,
                                     float* mod, cudaStream_t s);
 
+// The layer on host buffers, pipelined over row chunks (fh_host.cu).  Arguments
+// are validated by the caller; the workspace holds host_linear_workspace_bytes.
+size_t host_linear_workspace_bytes(int64_t K, int64_t N, int64_t chunk_rows);
+cudaError_t launch_nvfp4_linear_host(const uint16_t* x_host, int64_t M, int64_t K, float a_g, const uint8_t* w_codes,
+                                     const uint8_t* w_scales, float w_g, const uint16_t* bias, int64_t N,
+                                     uint16_t* y_host, unsigned long long* clip, int64_t chunk_rows, void* workspace,
+                                     cudaStream_t s, const char** why);
+
 }  // namespace fh

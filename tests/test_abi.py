@@ -134,6 +134,23 @@ def test_argument_validation_without_gpu(lib):
     assert d(fake, 8, 2688, fake, 16, P(24), None, 42, 16128, fake, fake, None) == 2  # proj misaligned
     assert d(fake, 8, 2688, fake, 16, fake, P(17), 42, 16128, fake, fake, None) == 2  # bias misaligned
     assert d(fake, 0, 2688, fake, 16, fake, None, 42, 16128, fake, fake, None) == 0   # no timesteps
+    hl = lib.fh_nvfp4_linear_host
+    hl.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_float, P, P, ctypes.c_float, P, ctypes.c_int64, P, P,
+                   ctypes.c_int64, P, ctypes.c_size_t, P]
+    wsb = lib.fh_nvfp4_linear_host_workspace_bytes
+    wsb.restype = ctypes.c_size_t
+    wsb.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
+    assert wsb(2688, 8064, 4096) > 0 and wsb(2688, 8064, 4000) == 0 and wsb(96, 8064, 4096) == 0
+    assert wsb(2688, 8060, 4096) == 0
+    need = wsb(2688, 8064, 4096)
+    ws = P(1 << 20)  # a 256-byte-aligned fake address (never dereferenced here)
+    assert hl(fake, 128, 2688, 1.0, fake, fake, 1.0, None, 8064, fake, None, 4000, ws, need, None) == 2  # chunk % 128
+    assert hl(fake, 128, 2688, 1.0, fake, fake, 1.0, None, 8064, fake, None, 4096, ws, need - 1, None) == 1
+    assert hl(fake, 128, 2688, 0.0, fake, fake, 1.0, None, 8064, fake, None, 4096, ws, need, None) == 1
+    assert hl(None, 128, 2688, 1.0, fake, fake, 1.0, None, 8064, fake, None, 4096, ws, need, None) == 1
+    assert hl(fake, 128, 2688, 1.0, fake, fake, 1.0, None, 8064, fake, None, 4096, P((1 << 20) + 16), need,
+              None) == 2  # workspace alignment
+    assert hl(fake, 0, 2688, 1.0, fake, fake, 1.0, None, 8064, fake, None, 4096, ws, need, None) == 0   # empty
     a = lib.fh_amax
     a.argtypes = [P, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, P, P]
     assert a(fake, 3, 5, 4, fake, None) == 2
