@@ -239,7 +239,10 @@ int fh_quantize_int8_rows(const uint16_t* x_dev, int64_t rows, int64_t d, int64_
  * every element written.  heads, tq, tk >= 0 (each below 2^31); d > 0,
  * d % 16 == 0, d <= 65536; tk % 4 == 0; q_dev, k_dev and s_dev 16-byte
  * aligned; sm_scale finite.  A bounded wait that expires sets the device error
- * word (fh_device_status) and the kernel drains and returns. */
+ * word (fh_device_status) and the kernel drains and returns.
+ * Environment: FH_INT8_TEST_STALL=1 (read at each launch) is a test hook that
+ * makes the first CTA's MMA warp stop before its first MMA, so the call ends
+ * with FH_ERR_TIMEOUT after about 4 s. */
 int fh_int8_attention_scores(const int8_t* q_dev, const float* q_scales_dev, const int8_t* k_dev,
                              const float* k_scales_dev, float sm_scale, float* s_dev, int64_t heads, int64_t tq,
                              int64_t tk, int64_t d, fh_stream_t stream);

@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "fh_internal.h"
 
@@ -291,6 +292,7 @@ struct ScoreParams {
   float sm_scale;
   int heads, tq, tk;
   int m_tiles, n_tiles, num_tiles, k_stages;
+  int stall;  // test hook: CTA 0's MMA warp stops before its first MMA (0: off)
 };
 
 struct RingI8 {
@@ -384,6 +386,12 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kTN);
       for (int kt = 0; kt < p.k_stages; ++kt) {
         if (!__all_sync(0xFFFFFFFFu, bar_wait(full_bar(st.slot), st.phase, abort_flag))) {
+          ok = false;
+          break;
+        }
+        if (p.stall && blockIdx.x == 0) {
+          // Test hook: stop without issuing or committing, so this CTA's
+          // producer and epilogue run into their bounded waits.
           ok = false;
           break;
         }
@@ -609,6 +617,8 @@ cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int
   p.n_tiles = (int)((tk + kTN - 1) / kTN);
   p.num_tiles = (int)heads * p.m_tiles * p.n_tiles;
   p.k_stages = (int)((d + kSK - 1) / kSK);  // the last stage's columns past d read as zero
+  const char* stall_env = getenv("FH_INT8_TEST_STALL");  // read at each launch
+  p.stall = (stall_env != nullptr && stall_env[0] == '1') ? 1 : 0;
   static int configured = -1;
   int dev = 0;
   cudaGetDevice(&dev);

@@ -146,3 +146,25 @@ def test_scores_full_size_sampled():
         h, i = divmod(int(flat), T)
         ref = oracle.int8_scores(q8[h:h + 1, i:i + 1], qs[h:h + 1, i:i + 1], k8[h:h + 1], ks[h:h + 1], sm_scale)
         _assert_scores(s[h:h + 1, i:i + 1], ref)
+
+
+def test_score_stall_times_out_drains_and_context_survives(monkeypatch):
+    """With the test hook FH_INT8_TEST_STALL=1 the first CTA's MMA warp stops
+    before its first MMA without committing; that CTA's producer and epilogue
+    run into their bounded waits (about 4 s), drain and free TMEM, and the host
+    reads FH_ERR_TIMEOUT.  With the hook off, scores in the same context pass."""
+    m = fh()
+    m.fh_device_status()
+    H, T, d = 2, 300, 128
+    q8 = torch.zeros((H, T, d), dtype=torch.int8, device="cuda")
+    qs = torch.ones((H, T), dtype=torch.float32, device="cuda")
+    s = torch.empty((H, T, T), dtype=torch.float32, device="cuda")
+    monkeypatch.setenv("FH_INT8_TEST_STALL", "1")
+    m.fh_int8_attention_scores(q8, qs, q8, qs, 1.0, s)
+    with pytest.raises(m.FHError) as e:
+        m.fh_device_status()
+    assert e.value.status == m.FH_ERR_TIMEOUT
+    monkeypatch.delenv("FH_INT8_TEST_STALL")
+    m.fh_device_status()  # the word was cleared
+    q8a, qsa, k8a, ksa, sm_scale, sa = _scores_case(2, 300, 260, 128, seed=11)
+    _assert_scores(sa, oracle.int8_scores(q8a, qsa, k8a, ksa, sm_scale))
