@@ -607,7 +607,7 @@ def bench_adaln(args):
 
 # DRAM bytes (read + write) of one int8_scores_kernel launch on the workload
 # above, from an ncu capture; valid only for the kernel source it was taken on.
-ATTN_TRAFFIC = {"bytes": 1371740416, "source_sha256": "dc7bc90db0be7c1e"}
+ATTN_TRAFFIC = {"bytes": 1371055104, "source_sha256": "5852781145a6cbf0"}
 
 
 def attn_traffic_valid():

@@ -237,7 +237,7 @@ int fh_quantize_int8_rows(const uint16_t* x_dev, int64_t rows, int64_t d, int64_
  * [heads, tq]; k_scales_dev FP32 [heads, tk] (the outputs of
  * fh_quantize_int8_rows over the flattened rows); s_dev: FP32 [heads, tq, tk],
  * every element written.  heads, tq, tk >= 0 (each below 2^31); d > 0,
- * d % 16 == 0, d <= 65536; tk % 4 == 0; q_dev, k_dev and s_dev 16-byte
+ * d % 16 == 0, d <= 65536 (any tk; tk % 4 == 0 takes 16-byte stores); q_dev, k_dev and s_dev 16-byte
  * aligned; sm_scale finite.  A bounded wait that expires sets the device error
  * word (fh_device_status) and the kernel drains and returns.
  * Environment: FH_INT8_TEST_STALL=1 (read at each launch) is a test hook that

@@ -298,9 +298,8 @@ int fh_int8_attention_scores(const int8_t* q_dev, const float* q_scales_dev, con
   g_last_error[0] = 0;
   if (!isfinite(sm_scale))
     return fail(FH_ERR_INVALID_ARG, "fh_int8_attention_scores: sm_scale must be finite%s");
-  if (heads < 0 || tq < 0 || tk < 0 || d <= 0 || d % 16 != 0 || tk % 4 != 0)
-    return fail(FH_ERR_UNSUPPORTED_SHAPE,
-                "fh_int8_attention_scores: need heads, tq, tk >= 0, d > 0, d %% 16 == 0, tk %% 4 == 0%s");
+  if (heads < 0 || tq < 0 || tk < 0 || d <= 0 || d % 16 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_int8_attention_scores: need heads, tq, tk >= 0, d > 0, d %% 16 == 0%s");
   if (heads > 0x7FFFFFFF || tq > 0x7FFFFFFF || tk > 0x7FFFFFFF || d > 65536)
     return fail(FH_ERR_UNSUPPORTED_SHAPE,
                 "fh_int8_attention_scores: heads, tq, tk must fit in 31 bits and d <= 65536%s");

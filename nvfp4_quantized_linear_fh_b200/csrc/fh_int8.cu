@@ -490,15 +490,23 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
               make_float4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
         }
         __syncwarp();
-        const int gcol = n0 + c * kOutCols + 4 * (lane & 7);  // tk % 4 == 0: a float4 never straddles tk
+        const int gcol = n0 + c * kOutCols + 4 * (lane & 7);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int r = 4 * i + (lane >> 3);
           const float4 val =
               *reinterpret_cast<const float4*>(sb + r * 128 + (((uint32_t)(lane & 7) ^ (uint32_t)(r & 7)) * 16));
           const int grow = m0 + 32 * q + r;
-          if (grow < p.tq && gcol < p.tk)
-            *reinterpret_cast<float4*>(p.out + ((size_t)h * p.tq + grow) * p.tk + gcol) = val;
+          if (grow >= p.tq) continue;
+          float* dst = p.out + ((size_t)h * p.tq + grow) * p.tk + gcol;
+          if ((p.tk & 3) == 0) {  // 16-byte rows: a float4 never straddles tk
+            if (gcol < p.tk) *reinterpret_cast<float4*>(dst) = val;
+          } else {  // any tk: element stores, each bounded
+            if (gcol < p.tk) dst[0] = val.x;
+            if (gcol + 1 < p.tk) dst[1] = val.y;
+            if (gcol + 2 < p.tk) dst[2] = val.z;
+            if (gcol + 3 < p.tk) dst[3] = val.w;
+          }
         }
         __syncwarp();  // the buffer is rewritten by the next chunk
       };

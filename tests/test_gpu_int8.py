@@ -99,7 +99,8 @@ def _assert_scores(s, ref):
 
 
 @pytest.mark.parametrize("H,tq,tk,d", [(1, 1, 4, 16), (3, 200, 300, 128), (2, 130, 516, 256), (2, 257, 260, 64),
-                                       (1, 128, 256, 144), (4, 333, 1000, 128), (1, 600, 4, 32)])
+                                       (1, 128, 256, 144), (4, 333, 1000, 128), (1, 600, 4, 32),
+                                       (2, 77, 301, 128), (1, 5, 1, 16), (3, 129, 258, 64)])
 def test_scores_match_oracle(H, tq, tk, d):
     q8, qs, k8, ks, sm_scale, s = _scores_case(H, tq, tk, d, seed=tq)
     _assert_scores(s, oracle.int8_scores(q8, qs, k8, ks, sm_scale))
