@@ -306,6 +306,9 @@ struct RingI8 {
   }
 };
 
+// kAligned: Tk % 4 == 0, so the rows of S are 16-byte aligned and every store
+// is a float4; otherwise element stores, each bounded.
+template <bool kAligned>
 __global__ void __launch_bounds__(kThreadsI8, 1)
     int8_scores_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const ScoreParams p) {
@@ -497,15 +500,17 @@ __global__ void __launch_bounds__(kThreadsI8, 1)
           const float4 val =
               *reinterpret_cast<const float4*>(sb + r * 128 + (((uint32_t)(lane & 7) ^ (uint32_t)(r & 7)) * 16));
           const int grow = m0 + 32 * q + r;
-          if (grow >= p.tq) continue;
-          float* dst = p.out + ((size_t)h * p.tq + grow) * p.tk + gcol;
-          if ((p.tk & 3) == 0) {  // 16-byte rows: a float4 never straddles tk
-            if (gcol < p.tk) *reinterpret_cast<float4*>(dst) = val;
-          } else {  // any tk: element stores, each bounded
-            if (gcol < p.tk) dst[0] = val.x;
-            if (gcol + 1 < p.tk) dst[1] = val.y;
-            if (gcol + 2 < p.tk) dst[2] = val.z;
-            if (gcol + 3 < p.tk) dst[3] = val.w;
+          if constexpr (kAligned) {  // a float4 never straddles tk
+            if (grow < p.tq && gcol < p.tk)
+              *reinterpret_cast<float4*>(p.out + ((size_t)h * p.tq + grow) * p.tk + gcol) = val;
+          } else {
+            if (grow < p.tq) {
+              float* dst = p.out + ((size_t)h * p.tq + grow) * p.tk + gcol;
+              if (gcol < p.tk) dst[0] = val.x;
+              if (gcol + 1 < p.tk) dst[1] = val.y;
+              if (gcol + 2 < p.tk) dst[2] = val.z;
+              if (gcol + 3 < p.tk) dst[3] = val.w;
+            }
           }
         }
         __syncwarp();  // the buffer is rewritten by the next chunk
@@ -631,12 +636,17 @@ cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(int8_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemI8);
+    cudaError_t e = cudaFuncSetAttribute(int8_scores_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemI8);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(int8_scores_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemI8);
     if (e != cudaSuccess) return e;
     configured = dev;
   }
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
-  int8_scores_kernel<<<grid, kThreadsI8, kSmemI8, s>>>(tmQ, tmK, p);
+  if (tk % 4 == 0)
+    int8_scores_kernel<true><<<grid, kThreadsI8, kSmemI8, s>>>(tmQ, tmK, p);
+  else
+    int8_scores_kernel<false><<<grid, kThreadsI8, kSmemI8, s>>>(tmQ, tmK, p);
   return cudaGetLastError();
 }
 
