@@ -607,7 +607,7 @@ def bench_adaln(args):
 
 # DRAM bytes (read + write) of one int8_scores_kernel launch on the workload
 # above, from an ncu capture; valid only for the kernel source it was taken on.
-ATTN_TRAFFIC = {"bytes": 1371055104, "source_sha256": "5852781145a6cbf0"}
+ATTN_TRAFFIC = {"bytes": 1371787776, "source_sha256": "1c5edf861590e2be"}
 
 
 def attn_traffic_valid():
