@@ -9,6 +9,8 @@ The calibration, the weight quantization and the input generation happen
 before the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fh|reference]
+  python bench.py --workload ffn|attn|adaln   (the FFN block, INT8 attention
+      scores and AdaLN basis projection, one GPU; secondary lines)
 
 With N > 1 (launched by torch.distributed.run) every rank runs the same
 per-GPU workload on its own GPU (rows of the token batch are independent:
