@@ -49,3 +49,45 @@ def test_weights_and_bias_distributions():
     b = S.bf16_to_f32(S.bias(layer))
     assert w.shape == (256, 256) and b.shape == (256,)
     assert abs(w.std() - 0.02) < 0.002 and abs(b.std() - 0.01) < 0.003
+
+
+def test_f16_rounding_matches_torch():
+    rng = np.random.default_rng(1)
+    x = np.concatenate([rng.standard_normal(20000) * 10.0 ** rng.integers(-8, 5, 20000),
+                        [0.0, -0.0, 1.0, 65504.0, 65520.0, 2.0 ** -24, 2.0 ** -25, 1.0 + 2.0 ** -11]])
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    with np.errstate(over="ignore"):                            # 65520 rounds to +inf on purpose
+        np.testing.assert_array_equal(S.to_f16_bits(x.astype(np.float32)), ref)
+
+
+def test_attention_qk_structure():
+    """Per-(head, channel) spreads, about one outlier channel in 32 at 8x, every
+    tenth token at 4x; queries and keys differ, the same call repeats."""
+    h, t, d = 4, 400, 256
+    q = S.attention_qk(h, t, d, "q")
+    assert q.shape == (h, t, d) and q.dtype == np.uint16
+    np.testing.assert_array_equal(q, S.attention_qk(h, t, d, "q"))
+    assert not np.array_equal(q, S.attention_qk(h, t, d, "k"))
+    v = S.bf16_to_f32(q).astype(np.float64)
+    body = np.delete(v, np.arange(0, t, 10), axis=1)
+    ch_std = body.std(axis=1)                                   # [h, d]
+    loud = ch_std > 8.0 * np.median(ch_std)
+    assert 0 < loud.sum() < h * d // 8
+    tenth = v[:, ::10, :]
+    ratio = np.abs(tenth).mean() / np.abs(body).mean()
+    assert 3.0 < ratio < 5.0
+
+
+def test_adaln_inputs_shapes_and_spreads():
+    e, basis, proj, bias = S.adaln_inputs(3, 500, 2688, 16, S.SAMPLER_TIMESTEPS, seed=2)
+    assert e.shape == (8, 2688) and basis.shape == (16, 2688)
+    assert proj.shape == (3, 500, 16) and bias.shape == (3, 500)
+    f16 = lambda b: b.view(np.float16).astype(np.float64)  # noqa: E731
+    assert abs(S.bf16_to_f32(e).std() - 1.0) < 0.05
+    assert np.allclose(np.linalg.norm(f16(basis), axis=1), 1.0, atol=0.05)
+    assert abs(f16(proj).std() - 0.05) < 0.005 and abs(f16(bias).std() - 0.01) < 0.002
+    # One seeded embedding per timestep: the same timestep gives the same row.
+    e2, *_ = S.adaln_inputs(1, 1, 2688, 16, (125, 999), seed=2)
+    np.testing.assert_array_equal(e2, e[[7, 0]])
+    e0, *_ = S.adaln_inputs(1, 1, 64, 16, ())
+    assert e0.shape == (0, 64)
