@@ -31,6 +31,13 @@
  *     stream) and the call returns without synchronizing, except where stated.
  *   - The return value is an fh_status.  On failure nothing was enqueued and
  *     fh_last_error() (per host thread) describes the cause.
+ *   - Host threads: the property caches are filled by the first call of each
+ *     entry point on a device and only read afterwards.  With one device per
+ *     process (the intended deployment, one process per GPU), make that first
+ *     call from one thread; later calls may come from several threads at once.
+ *     A process that drives several devices must serialize its calls, since
+ *     the caches hold the most recent device.  fh_nvfp4_linear_host keeps its
+ *     copy stream per host thread.
  *   - Matrices are row-major.  BF16 values are passed as their uint16 bits.
  *   - Inputs must be finite; results for NaN or Inf inputs are unspecified.
  */
