@@ -1,7 +1,9 @@
 """The multi-GPU host path with two gloo ranks on CPU: row sharding,
 calibration amax all-reduce, clip-count sum and max-over-ranks timing.  The
 per-rank arithmetic is the oracle's (no GPU here); the point is that sharded
-calibration and quantization reproduce the unsharded results exactly."""
+calibration and quantization reproduce the unsharded results exactly, and that
+the INT8 attention scores (by head) and the AdaLN projection (by timestep and
+by block) split into replicas whose shares reassemble the unsharded result."""
 import os
 import socket
 
@@ -81,3 +83,55 @@ def test_shard_rows_partitions():
                 assert all(a % align == 0 for a, b in spans if b > a)
     with pytest.raises(ValueError):
         shard_rows(10, 2, 2)
+
+
+def _replica_worker(rank, world, port, out_dir):
+    """The secondary workloads as replicas: attention scores split by head, AdaLN
+    codes by timestep and modulations by block, each rank computing its share
+    with no exchange in the data path (only the barrier the bench takes)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import oracle
+    import synthetic as S
+    from nvfp4_quantized_linear_fh_b200 import dist as fhd
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        H, T, d = 5, 40, 32
+        q = S.attention_qk(H, T, d, "q", seed=7)
+        k = S.attention_qk(H, T, d, "k", seed=7)
+        h0, h1 = fhd.shard_rows(H, world, rank)
+        q8, qs = oracle.quantize_int8_rows(q[h0:h1].reshape(-1, d))
+        k8, ks = oracle.quantize_int8_rows(k[h0:h1].reshape(-1, d))
+        n = h1 - h0
+        s = oracle.int8_scores(q8.reshape(n, T, d), qs.reshape(n, T), k8.reshape(n, T, d), ks.reshape(n, T),
+                               d ** -0.5)
+        e, basis, proj, bias = S.adaln_inputs(3, 24, 64, 16, S.SAMPLER_TIMESTEPS, seed=5)
+        t0, t1 = fhd.shard_rows(e.shape[0], world, rank)
+        code = oracle.adaln_code(e[t0:t1], basis)
+        l0, l1 = fhd.shard_rows(proj.shape[0], world, rank)
+        mod = oracle.adaln_modulation(oracle.adaln_code(e, basis), proj[l0:l1], bias[l0:l1])
+        dist.barrier()
+        np.savez(os.path.join(out_dir, f"replica{rank}.npz"), s=s, code=code, mod=mod)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2])
+def test_secondary_workloads_shard_without_exchange(tmp_path, world):
+    import oracle
+    import synthetic as S
+    mp.spawn(_replica_worker, args=(world, free_port(), str(tmp_path)), nprocs=world, join=True)
+    parts = [np.load(tmp_path / f"replica{r}.npz") for r in range(world)]
+    H, T, d = 5, 40, 32
+    q8, qs = oracle.quantize_int8_rows(S.attention_qk(H, T, d, "q", seed=7).reshape(-1, d))
+    k8, ks = oracle.quantize_int8_rows(S.attention_qk(H, T, d, "k", seed=7).reshape(-1, d))
+    s_ref = oracle.int8_scores(q8.reshape(H, T, d), qs.reshape(H, T), k8.reshape(H, T, d), ks.reshape(H, T),
+                               d ** -0.5)
+    np.testing.assert_array_equal(np.concatenate([p["s"] for p in parts]), s_ref)
+    e, basis, proj, bias = S.adaln_inputs(3, 24, 64, 16, S.SAMPLER_TIMESTEPS, seed=5)
+    code_ref = oracle.adaln_code(e, basis)
+    np.testing.assert_array_equal(np.concatenate([p["code"] for p in parts]), code_ref)
+    np.testing.assert_array_equal(np.concatenate([p["mod"] for p in parts]),
+                                  oracle.adaln_modulation(code_ref, proj, bias))
