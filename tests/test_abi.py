@@ -141,6 +141,11 @@ def test_argument_validation_without_gpu(lib):
     wsb.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int64]
     assert wsb(2688, 8064, 4096) > 0 and wsb(2688, 8064, 4000) == 0 and wsb(96, 8064, 4096) == 0
     assert wsb(2688, 8060, 4096) == 0
+    # The workspace holds two BF16 x slots, one chunk of codes and MMA-tiled
+    # scales, and two BF16 y slots, each padded to 256 bytes at most.
+    for K, N, chunk in [(2688, 8064, 4096), (64, 8, 128), (2688, 10752, 1024), (10752, 2688, 384), (192, 24, 256)]:
+        raw = 2 * chunk * K * 2 + chunk * K // 2 + -(-chunk // 128) * 128 * -(-(K // 16) // 4) * 4 + 2 * chunk * N * 2
+        assert raw <= wsb(K, N, chunk) <= raw + 6 * 255, (K, N, chunk)
     need = wsb(2688, 8064, 4096)
     ws = P(1 << 20)  # a 256-byte-aligned fake address (never dereferenced here)
     assert hl(fake, 128, 2688, 1.0, fake, fake, 1.0, None, 8064, fake, None, 4000, ws, need, None) == 2  # chunk % 128
