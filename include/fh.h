@@ -31,13 +31,13 @@
  *     stream) and the call returns without synchronizing, except where stated.
  *   - The return value is an fh_status.  On failure nothing was enqueued and
  *     fh_last_error() (per host thread) describes the cause.
- *   - Host threads: the property caches are filled by the first call of each
- *     entry point on a device and only read afterwards.  With one device per
- *     process (the intended deployment, one process per GPU), make that first
- *     call from one thread; later calls may come from several threads at once.
- *     A process that drives several devices must serialize its calls, since
- *     the caches hold the most recent device.  fh_nvfp4_linear_host keeps its
- *     copy stream per host thread.
+ *   - Host threads: the property caches are per-device tables of atomics,
+ *     filled by the first call of an entry point on each device (with that
+ *     device current) and only read afterwards, so calls may come from several
+ *     host threads at once and a process may drive several devices (up to 64
+ *     device ordinals are cached; higher ones are served uncached).  The
+ *     quantizer's decision tables are cached per host thread.
+ *     fh_nvfp4_linear_host keeps its copy streams per host thread and device.
  *   - Matrices are row-major.  BF16 values are passed as their uint16 bits.
  *   - Inputs must be finite; results for NaN or Inf inputs are unspecified.
  */
@@ -191,14 +191,24 @@ int fh_nvfp4_linear_gelu_quant(const uint8_t* a_codes_dev, const uint8_t* a_scal
  * pageable memory works, but then the copies do not overlap.  Weights, bias and
  * the clip counter (may be NULL) are device memory as in fh_nvfp4_linear.
  * The rows are processed in chunks of chunk_rows (a multiple of 128): each
- * chunk's upload, quantization and GEMM run on `stream` while the previous
- * chunk's download runs on a copy stream the library keeps per host thread and
- * device, so transfers in both directions and the kernels overlap.  The call
- * is ordered on `stream` like any other: work enqueued there afterwards sees
- * y_host complete (synchronize before reading it on the host).
+ * chunk's quantization and GEMM run on `stream`, while the next chunk's upload
+ * and the previous chunk's download run on two copy streams, so transfers in
+ * both directions and the kernels overlap.  The call is ordered on `stream`
+ * like any other: the copies start after the work enqueued there before the
+ * call, and work enqueued there afterwards sees y_host complete (synchronize
+ * before reading it on the host).
  * workspace_dev: device memory owned by the caller, 256-byte aligned, at least
  * fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows) bytes (two x chunks,
- * the chunk's codes and scales, two y chunks); the library allocates none.
+ * the chunk's codes and scales, two y chunks), not used by other work while
+ * the call runs; the library allocates no device memory.  The exception to the
+ * "allocates nothing" convention: on the first call from a host thread on a
+ * device, the library creates that thread's two copy streams and eleven events
+ * for the device, kept until the process exits.
+ * Failure: argument errors enqueue nothing.  A CUDA error in the middle of the
+ * chunk loop returns FH_ERR_CUDA after part of the work was enqueued; that
+ * work stays ordered on `stream` (the copy streams are joined back into it
+ * before the call returns), so synchronize `stream` before freeing x_host,
+ * y_host or the workspace.
  * Shape rules as fh_nvfp4_linear (K % 64 == 0, N % 8 == 0). */
 int fh_nvfp4_linear_host(const uint16_t* x_host, int64_t M, int64_t K, float a_gscale, const uint8_t* w_codes_dev,
                          const uint8_t* w_scales_dev, float w_gscale, const uint16_t* bias_dev, int64_t N,

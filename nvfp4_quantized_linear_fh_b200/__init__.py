@@ -262,12 +262,19 @@ def fh_nvfp4_linear_host(x_host: torch.Tensor, a_gscale: float, w_codes: torch.T
     if clip is not None and (clip.dtype != torch.int64 or clip.device.type != "cuda"):
         raise TypeError("clip must be a CUDA int64 tensor")
     need = fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows)
-    if workspace is None:
+    own = workspace is None
+    if own:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=w_codes.device)
     _need(workspace, _U8, "workspace")
+    torch_stream = torch.cuda.current_stream(w_codes.device) if stream is None else stream
     _check(_lib.fh_nvfp4_linear_host(_P(x_host.data_ptr()), M, K, float(a_gscale), _ptr(w_codes), _ptr(w_scales),
                                      float(w_gscale), _ptr(bias), N, _P(y_host.data_ptr()), _ptr(clip), chunk_rows,
-                                     _ptr(workspace), workspace.numel(), _stream(stream)))
+                                     _ptr(workspace), workspace.numel(), _stream(torch_stream)))
+    if own:
+        # The call's work on `stream` still uses the workspace after this returns:
+        # the caching allocator must not hand the block to other streams before
+        # that work has finished.
+        workspace.record_stream(torch_stream)
 
 
 def fh_scales_to_rowmajor(tiled: torch.Tensor, rowmajor: torch.Tensor, rows: int, K: int, stream=None) -> None:
