@@ -200,12 +200,15 @@ cudaError_t launch_mod(const uint16_t* proj, const uint16_t* bias, const float* 
                        int64_t n, float* mod, cudaStream_t s) {
   const int64_t rows_total = L * n;
   const int64_t groups = (rows_total + (int64_t)kModThreads * kModRows - 1) / ((int64_t)kModThreads * kModRows);
-  static int per_sm = 0;  // resident CTAs per SM for this instantiation (one wave)
-  if (per_sm == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, adaln_mod_kernel<RC>, kModThreads, 0);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) per_sm = 1;
-  }
+  static DeviceTable resident;  // resident CTAs per SM for this instantiation (one wave)
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int per_sm = per_device(resident, dev, [](int) {
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, adaln_mod_kernel<RC>, kModThreads, 0);
+    return e != cudaSuccess ? -(int)e : (n < 1 ? 1 : n);
+  });
+  if (per_sm <= 0) return (cudaError_t)(-per_sm);
   const int64_t cap = (int64_t)sm_count() * per_sm;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(groups < cap ? groups : cap));

@@ -27,17 +27,17 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Device checks shared by every entry point: a current device of compute
 // capability 10.0 (B200 class).  Cached per device.
 int check_device() {
-  static int checked_dev = -1;
+  static fh::DeviceTable checked;
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev == checked_dev) return FH_OK;
-  int major = 0, minor = 0;
-  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-  if (major != 10 || minor != 0)
-    return fail(FH_ERR_NO_DEVICE, "current device is not an sm_100 GPU%s");
-  checked_dev = dev;
+  const int ok = fh::per_device(checked, dev, [](int d) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, d);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, d);
+    return (major == 10 && minor == 0) ? 1 : -1;
+  });
+  if (ok <= 0) return fail(FH_ERR_NO_DEVICE, "current device is not an sm_100 GPU%s");
   return FH_OK;
 }
 
@@ -46,13 +46,14 @@ int check_device() {
 namespace fh {
 
 int sm_count() {
-  static int dev_cached = -1, count = 0;
+  static DeviceTable counts;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev != dev_cached) {
-    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-    dev_cached = dev;
-  }
+  const int count = per_device(counts, dev, [](int d) {
+    int c = 0;
+    cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, d);
+    return c;
+  });
   return count > 0 ? count : 1;
 }
 

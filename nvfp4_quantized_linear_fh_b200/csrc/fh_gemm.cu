@@ -8,8 +8,8 @@
 // runs": the RTX 4090 lacks FP4 tensor cores, Blackwell has them).
 //
 // Design: persistent, warp-specialized, one CTA per SM.  By default two CTAs
-// of a cluster pair up on one 256 x 192 output tile with tcgen05.mma
-// cta_group::2 (each SM computes 128 rows; the 192 W rows are split 96/96
+// of a cluster pair up on one 256 x 256 output tile with tcgen05.mma
+// cta_group::2 (each SM computes 128 rows; the 256 W rows are split 128/128
 // between the two SMs' shared memory, so each SM loads and holds half of W);
 // the single-CTA form (128 x 192 tiles) is the same code with kCta = 1.
 // Two tile forms (template parameter BN):
@@ -835,14 +835,15 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (fn == nullptr) {
+  // Looked up once per process (thread-safe static initialization).
+  static const EncodeTiledFn fn = []() -> EncodeTiledFn {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
+      return reinterpret_cast<EncodeTiledFn>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -858,22 +859,20 @@ int stall_group() {
 // environment variable FH_GEMM_CTAS=1 selects the single-CTA form (both run the
 // same arithmetic; the switch exists to compare them).
 int cta_mode() {
-  static int mode = 0;
-  if (mode == 0) {
+  static const int mode = []() {
     const char* e = getenv("FH_GEMM_CTAS");
-    mode = (e != nullptr && e[0] == '1') ? 1 : 2;
-  }
+    return (e != nullptr && e[0] == '1') ? 1 : 2;
+  }();
   return mode;
 }
 
 // Tile width of the CTA-pair form for an N-column output: 256 unless the
 // environment variable FH_GEMM_BN (read at first launch) is 192.
 int tile_width(int64_t N) {
-  static int forced = -1;
-  if (forced < 0) {
+  static const int forced = []() {
     const char* e = getenv("FH_GEMM_BN");
-    forced = (e != nullptr && strcmp(e, "192") == 0) ? 192 : (e != nullptr && strcmp(e, "256") == 0) ? 256 : 0;
-  }
+    return (e != nullptr && strcmp(e, "192") == 0) ? 192 : (e != nullptr && strcmp(e, "256") == 0) ? 256 : 0;
+  }();
   if (forced != 0) return forced;
   (void)N;
   return 256;
@@ -884,15 +883,14 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
                         const CUtensorMap& tmSB, const CUtensorMap& tmY, const Params& p,
                         const typename EpiSel<kEpi>::type& eq, cudaStream_t s) {
   using C = Cfg<kCta, kBN>;
-  static int configured_device = -1;
-  static int max_groups = 0;
+  static DeviceTable groups_of;  // resident CTA groups of this form, per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_device != dev) {
+  const int max_groups = per_device(groups_of, dev, [](int) {
     cudaError_t e =
         cudaFuncSetAttribute(nvfp4_linear_kernel<kCta, kEpi, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
-    if (e != cudaSuccess) return e;
-    max_groups = sm_count() / kCta;
+    if (e != cudaSuccess) return -(int)e;
+    int max_groups = sm_count() / kCta;
     if (kCta == 2) {
       // Clusters that fit at once (an SM left without a partner cannot host one).
       cudaLaunchConfig_t cfg = {};
@@ -912,8 +910,9 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
         max_groups = clusters < max_groups ? clusters : max_groups;
       cudaGetLastError();
     }
-    configured_device = dev;
-  }
+    return max_groups > 0 ? max_groups : 1;
+  });
+  if (max_groups <= 0) return (cudaError_t)(-max_groups);
   const int groups = p.num_tiles < max_groups ? p.num_tiles : max_groups;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];

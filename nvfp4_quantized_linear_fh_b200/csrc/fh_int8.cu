@@ -553,14 +553,15 @@ typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void
                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeFn encode3() {
-  static EncodeFn fn = nullptr;
-  if (fn == nullptr) {
+  // Looked up once per process (thread-safe static initialization).
+  static const EncodeFn fn = []() -> EncodeFn {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(ptr);
-  }
+      return reinterpret_cast<EncodeFn>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -632,16 +633,16 @@ cudaError_t launch_int8_scores(const int8_t* q, const float* q_scales, const int
   p.k_stages = (int)((d + kSK - 1) / kSK);  // the last stage's columns past d read as zero
   const char* stall_env = getenv("FH_INT8_TEST_STALL");  // read at each launch
   p.stall = (stall_env != nullptr && stall_env[0] == '1') ? 1 : 0;
-  static int configured = -1;
+  static DeviceTable configured;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured != dev) {
+  const int cfg = per_device(configured, dev, [](int) {
     cudaError_t e = cudaFuncSetAttribute(int8_scores_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemI8);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(int8_scores_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemI8);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+    return e == cudaSuccess ? 1 : -(int)e;
+  });
+  if (cfg <= 0) return (cudaError_t)(-cfg);
   const int grid = p.num_tiles < sm_count() ? p.num_tiles : sm_count();
   if (tk % 4 == 0)
     int8_scores_kernel<true><<<grid, kThreadsI8, kSmemI8, s>>>(tmQ, tmK, p);

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/fh.h"
 #include "fh_nvfp4.cuh"
 
@@ -23,6 +25,28 @@ cudaError_t read_and_clear_quant_error(unsigned int* bits);
 
 // The INT8 score kernel's error word (fh_int8.cu); call after the stream is synchronized.
 cudaError_t read_and_clear_int8_error(unsigned int* bits);
+
+// Per-device caches of the host side.  Each table holds one int per device
+// ordinal, 0 meaning "not filled yet"; the first call on a device fills its
+// entry with the device current.  Entries are atomics, so host threads may
+// race on the first fill: each computes the same value and the last store
+// wins.  Devices beyond the table are served uncached.
+constexpr int kMaxDevices = 64;
+using DeviceTable = std::atomic<int>[kMaxDevices];
+
+// The value for device `dev` from `table`, computing it with fill(dev) on the
+// first use.  fill returns a value > 0, or <= 0 for a failure, which is
+// returned without being cached.
+template <class F>
+int per_device(DeviceTable& table, int dev, F fill) {
+  if (dev < 0 || dev >= kMaxDevices) return fill(dev);
+  int v = table[dev].load(std::memory_order_acquire);
+  if (v == 0) {
+    v = fill(dev);
+    if (v > 0) table[dev].store(v, std::memory_order_release);
+  }
+  return v;
+}
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
