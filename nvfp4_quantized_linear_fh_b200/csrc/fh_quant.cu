@@ -265,6 +265,17 @@ __device__ __forceinline__ bool q_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// L2 policy of the loads of x: every byte of x is read exactly once, so its
+// lines are the first candidates for eviction.  Lines that other kernels left
+// in L2 -- notably the preceding GEMM's output, still dirty -- then stay there
+// instead of being written back while this kernel streams x; their write-back
+// happens later, under the next GEMM, which leaves HBM bandwidth to spare.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // Bounded wait (about 4 s, or until another warp of the CTA gave up).
 __device__ __forceinline__ bool q_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (q_try_wait(bar, parity)) return true;
@@ -339,6 +350,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
   if (warp == kQConsumerWarps) {
     // ===== producer: bulk copies of whole units into the stage ring =====
     if (lane == 0) {
+      const uint64_t read_once = evict_first_policy();
       int st = 0;
       uint32_t ph = 0;
       for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
@@ -355,15 +367,16 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
                      : "memory");
         if (p.one_copy) {
           asm volatile(
-              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-              "l"(src), "r"((uint32_t)rows * row_bytes), "r"(full_bar(st))
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+              " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+              "l"(src), "r"((uint32_t)rows * row_bytes), "r"(full_bar(st)), "l"(read_once)
               : "memory");
         } else {
           for (int64_t r = 0; r < rows; ++r)
             asm volatile(
-                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                    dst + (uint32_t)r * row_bytes),
-                "l"(src + r * p.ldx), "r"(row_bytes), "r"(full_bar(st))
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+                " [%0], [%1], %2, [%3], %4;" ::"r"(dst + (uint32_t)r * row_bytes),
+                "l"(src + r * p.ldx), "r"(row_bytes), "r"(full_bar(st)), "l"(read_once)
                 : "memory");
         }
         if (++st == kQStages) {
@@ -472,6 +485,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
   if (warp == kQConsumerWarps) {
     // ===== producer: one tensor TMA per 128 x 64 tile =====
     if (lane == 0) {
+      const uint64_t read_once = evict_first_policy();
       int st = 0;
       uint32_t ph = 0;
       int tr = row0, tc = col0;
@@ -488,9 +502,9 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
                      "r"((uint32_t)kQUnitBytes)
                      : "memory");
         asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-            " [%0], [%1, {%2, %3}], [%4];" ::"r"(stage0 + st * kQUnitBytes),
-            "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(x0), "r"(y0), "r"(full_bar(st))
+            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+            " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(stage0 + st * kQUnitBytes),
+            "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(x0), "r"(y0), "r"(full_bar(st)), "l"(read_once)
             : "memory");
         if (++st == kQStages) {
           st = 0;
@@ -676,18 +690,23 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   const bool gather4 = (K / 16) % 4 == 0;
   const int64_t want = p.n_units > 0 ? p.n_units : 1;
   const int grid = (int)(want < 2 * (int64_t)sm_count() ? want : 2 * (int64_t)sm_count());
-  auto launch = [&](auto kernel, int& configured) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured != dev) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  // Shared-memory opt-in of a kernel, once per device.
+  auto configure = [&](auto kernel, DeviceTable& table) {
+    const int v = per_device(table, dev, [&](int) {
       cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
-      if (e != cudaSuccess) return e;
-      configured = dev;
-    }
+      return e == cudaSuccess ? 1 : -(int)e;
+    });
+    return v > 0 ? cudaSuccess : (cudaError_t)(-v);
+  };
+  auto launch = [&](auto kernel, DeviceTable& table) {
+    cudaError_t e = configure(kernel, table);
+    if (e != cudaSuccess) return e;
     kernel<<<grid, kQThreads, kQSmem, s>>>(p);
     return cudaGetLastError();
   };
-  static int cfg_ft = -1, cfg_ff = -1;
+  static DeviceTable cfg_ft, cfg_ff, cfg_t[2];
   if (tiled) {
     // K % 64 == 0 here.  One unit per 128-row x 64-column tile.
     CUtensorMap tmx;
@@ -697,15 +716,9 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
     p.n_units = ((M + 127) / 128) * (K / 64);
     const int64_t tw = p.n_units > 0 ? p.n_units : 1;
     const int tgrid = (int)(tw < 2 * (int64_t)sm_count() ? tw : 2 * (int64_t)sm_count());
-    static int cfg_t[2] = {-1, -1};
-    int dev = 0;
-    cudaGetDevice(&dev);
     auto kernel = gelu ? quantize_tiled_kernel<true> : quantize_tiled_kernel<false>;
-    if (cfg_t[gelu] != dev) {
-      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQSmem);
-      if (e != cudaSuccess) return e;
-      cfg_t[gelu] = dev;
-    }
+    cudaError_t e = configure(kernel, cfg_t[gelu ? 1 : 0]);
+    if (e != cudaSuccess) return e;
     kernel<<<tgrid, kQThreads, kQSmem, s>>>(tmx, p);
     return cudaGetLastError();
   }
