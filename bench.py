@@ -703,6 +703,11 @@ def main():
     achieved = r["flops"] / gemm_mean / 1e12
     fp4_sust = pk["bf16_sustained"] * FP4_OVER_BF16
     fp4_burst = pk["bf16"] * FP4_OVER_BF16
+    # The denominator matches the regime of the timed region: a region under a
+    # second runs before the power limit settles the clocks (the burst GEMM
+    # figure); a longer one runs at the power-capped clocks (the sustained one).
+    sustained = r["t_step"] >= 1.0
+    fp4_peak = fp4_sust if sustained else fp4_burst
     quant_gbs = QUANT_BYTES_PER_ELEM * r["M"] * r["K"] / quant_mean / 1e9
     e2e_value = r["flops"] * r["e_steps"] * world / r["t_e2e"] / 1e12 if r["e_steps"] else None
     line = {
@@ -712,9 +717,13 @@ def main():
         "data": "synthetic (seeded; calibrated per-layer scale; random-init weights)", "config": cfg,
         "gpu_launches": 2 * K_steps,
         "roofline": {"kernel": "nvfp4_linear_kernel", "bound": "tensor", "achieved": achieved,
-                     "peak": fp4_sust, "unit": "TFLOP/s", "frac": achieved / fp4_sust,
-                     "peak_note": f"{pk['source']} bf16 sustained {pk['bf16_sustained']} x 4 (nominal FP4/BF16)",
+                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                     "peak_note": (f"{pk['source']} bf16 {'sustained' if sustained else 'burst'} "
+                                   f"{pk['bf16_sustained'] if sustained else pk['bf16']} x 4 (nominal FP4/BF16); "
+                                   f"timed region {r['t_step']:.3f} s "
+                                   f"({'>=' if sustained else '<'} 1 s: {'sustained' if sustained else 'burst'})"),
                      "frac_of_burst_peak": achieved / fp4_burst,
+                     "frac_of_sustained_peak": achieved / fp4_sust,
                      "traffic": gemm_traffic() if r["M"] == WORKLOAD["M"] else None,
                      "traffic_note": "bytes per launch, ncu dram__bytes_read.sum + dram__bytes_write.sum",
                      "algorithmic_bytes": gemm_bytes(r["M"], r["N"], r["K"])},
