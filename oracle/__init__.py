@@ -59,6 +59,8 @@ def lib():
         L.oracle_quantize.restype = None
         L.oracle_quantize.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_int64, c.c_float,
                                       c.c_void_p, c.c_void_p, c.c_void_p]
+        L.oracle_clip_count.restype = c.c_uint64
+        L.oracle_clip_count.argtypes = [c.c_void_p, c.c_int64, c.c_int64, c.c_int64, c.c_float]
         L.oracle_linear.restype = None
         L.oracle_linear.argtypes = [c.c_void_p, c.c_void_p, c.c_float, c.c_void_p, c.c_void_p, c.c_float,
                                     c.c_void_p, c.c_int64, c.c_int64, c.c_void_p, c.c_int64,
@@ -130,6 +132,15 @@ def quantize(x_bits: np.ndarray, sg: float):
     clip = np.zeros(1, dtype=np.uint64)
     lib().oracle_quantize(_ptr(x), M, K, K, float(sg), _ptr(codes), _ptr(scales), _ptr(clip))
     return codes, scales, int(clip[0])
+
+
+def clip_count(x_bits: np.ndarray, sg: float) -> int:
+    """Number of elements of BF16 x (uint16 bits, any 2-D shape) with
+    |x| > 2688 * sg: the clip count of quantize(x, sg) without the codes."""
+    x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    return int(lib().oracle_clip_count(_ptr(x), x.shape[0], x.shape[1], x.shape[1], float(sg)))
 
 
 def tiled_scale_offsets(rows: int, K: int) -> np.ndarray:

@@ -134,30 +134,44 @@ float oracle_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld) {
 /* ---------------------------------------------------------------------- */
 
 /* Block scale: S_b = E4M3 RNE (saturating) of amax_b / (6 * s_g).
- * Compared as amax_b against mid * 6 * s_g, which is exact in binary64. */
-static int block_scale_code(double amax_b, double sg) {
-  int best = 0;
+ * Compared as amax_b against mid * 6 * s_g, which is exact in binary64; the
+ * boundaries t[c] = mid(c-1, c) * 6 * s_g depend on s_g only, so a call
+ * computes them once (scale_boundaries) and every block compares with them. */
+static void scale_boundaries(double sg, double t[E4M3_MAX_CODE + 1]) {
+  t[0] = 0.0;
   for (int c = 1; c <= E4M3_MAX_CODE; ++c) {
     double mid = 0.5 * (oracle_e4m3_value(c - 1) + oracle_e4m3_value(c));
-    double t = mid * FP4_MAX * sg;
-    if (amax_b > t || (amax_b == t && (c % 2) == 0)) best = c;
+    t[c] = mid * FP4_MAX * sg;
   }
+}
+
+static int block_scale_code(double amax_b, const double t[E4M3_MAX_CODE + 1]) {
+  int best = 0;
+  for (int c = 1; c <= E4M3_MAX_CODE; ++c)
+    if (amax_b > t[c] || (amax_b == t[c] && (c % 2) == 0)) best = c;
   return best;
 }
 
 /* Element code: sign bit = sign bit of x (so -0 and small negatives give 8);
  * magnitude = E2M1 RNE (saturating at 6) of |x| / (S_b * s_g), compared as
- * |x| against mid * S_b * s_g (exact in binary64).  S_b == 0 gives magnitude 0. */
-static int element_code(double x, double S, double sg) {
+ * |x| against mid * S_b * s_g (exact in binary64).  S_b == 0 gives magnitude
+ * 0.  The seven boundaries t[c] = mid(c-1, c) * S_b * s_g are the block's, so
+ * a block computes them once (element_boundaries). */
+static void element_boundaries(double S, double sg, double t[8]) {
+  t[0] = 0.0;
+  for (int c = 1; c <= 7; ++c) {
+    double mid = 0.5 * (oracle_e2m1_value(c - 1) + oracle_e2m1_value(c));
+    t[c] = mid * S * sg;
+  }
+}
+
+static int element_code(double x, double S, const double t[8]) {
   int sign = signbit(x) ? 8 : 0;
   double a = fabs(x);
   if (S == 0.0) return sign;
   int best = 0;
-  for (int c = 1; c <= 7; ++c) {
-    double mid = 0.5 * (oracle_e2m1_value(c - 1) + oracle_e2m1_value(c));
-    double t = mid * S * sg;
-    if (a > t || (a == t && (c % 2) == 0)) best = c;
-  }
+  for (int c = 1; c <= 7; ++c)
+    if (a > t[c] || (a == t[c] && (c % 2) == 0)) best = c;
   return sign | best;
 }
 
@@ -174,6 +188,8 @@ void oracle_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
   const double limit = FP4_MAX * E4M3_MAX * sg; /* exact */
   const int64_t nb = K / 16;
   uint64_t nclip = 0;
+  double st[E4M3_MAX_CODE + 1];
+  scale_boundaries(sg, st);
   /* Rows are independent; the clip count is an integer sum. */
 #pragma omp parallel for schedule(static) reduction(+ : nclip)
   for (int64_t m = 0; m < M; ++m) {
@@ -184,14 +200,16 @@ void oracle_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
         double a = fabs(oracle_bf16_value(row[16 * b + i]));
         if (a > amax) amax = a;
       }
-      int sc = block_scale_code(amax, sg);
+      int sc = block_scale_code(amax, st);
       double S = oracle_e4m3_value(sc);
+      double et[8];
+      element_boundaries(S, sg, et);
       scales[m * nb + b] = (uint8_t)sc;
       for (int i = 0; i < 16; i += 2) {
         double x0 = oracle_bf16_value(row[16 * b + i]);
         double x1 = oracle_bf16_value(row[16 * b + i + 1]);
-        int c0 = element_code(x0, S, sg);
-        int c1 = element_code(x1, S, sg);
+        int c0 = element_code(x0, S, et);
+        int c1 = element_code(x1, S, et);
         codes[m * (K / 2) + 8 * b + i / 2] = (uint8_t)(c0 | (c1 << 4));
         if (fabs(x0) > limit) ++nclip;
         if (fabs(x1) > limit) ++nclip;
@@ -199,6 +217,19 @@ void oracle_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
     }
   }
   *clip += nclip;
+}
+
+/* Clip count alone: the number of elements of x [M, K] (leading dimension
+ * ldx) with |x| > 2688 * sg, the largest magnitude the scaled format can
+ * represent (the same count oracle_quantize adds to *clip). */
+uint64_t oracle_clip_count(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float sg_f) {
+  const double limit = FP4_MAX * E4M3_MAX * (double)sg_f; /* exact */
+  uint64_t n = 0;
+#pragma omp parallel for schedule(static) reduction(+ : n)
+  for (int64_t m = 0; m < M; ++m)
+    for (int64_t k = 0; k < K; ++k)
+      if (fabs(oracle_bf16_value(x[m * ldx + k])) > limit) ++n;
+  return n;
 }
 
 /* Dequantize a quantized [rows, K] matrix row r into out[0..K): the E2M1 value

@@ -371,3 +371,21 @@ def test_gelu(oracle_mod):
         got = oracle_mod.gelu(S.to_bf16_bits(np.array([xv])))[0]
         bound = 945 / xv**10 * 1.01     # the next term of the alternating series
         assert abs(got - asym) <= abs(asym) * bound, (xv, got, asym)
+
+
+def test_clip_count_at_the_limit_and_by_brute_force(oracle_mod):
+    """clip_count counts |x| > 2688 s_g exactly: an element equal to the limit
+    is not clipped, the next BF16 above it is, in both signs; on random wide-
+    range inputs it equals a rational count and quantize()'s clip count."""
+    sg = 1.0 / 1024                       # limit 2688 / 1024 = 2.625, a BF16 value
+    lim = S.to_bf16_bits(np.array([2.625]))[0]
+    above = np.uint16(lim + 1)            # next BF16 magnitude up
+    below = np.uint16(lim - 1)
+    row = np.array([lim, above, below, lim | 0x8000, above | 0x8000, 0, 0x8000, below | 0x8000] * 2, dtype=np.uint16)
+    assert oracle_mod.clip_count(row, sg) == 4
+    assert oracle_mod.quantize(row.reshape(1, -1), sg)[2] == 4
+    rng = np.random.default_rng(5)
+    x = S.to_bf16_bits(rng.standard_normal((64, 128)) * np.exp(rng.uniform(-3, 3, (64, 1))))
+    for sg in (1e-3, 2.0 ** -12, float(np.float32(0.0037))):
+        want = sum(1 for v in S.bf16_to_f32(x).reshape(-1) if abs(Fraction(float(v))) > 2688 * Fraction(sg))
+        assert oracle_mod.clip_count(x, sg) == want == oracle_mod.quantize(x, sg)[2]
