@@ -266,3 +266,123 @@ def adaln_inputs(blocks: int, n: int, d: int, r: int, timesteps, seed: int = 0):
     proj = normal(derive_seed("adaln-proj", seed, blocks, n, r), 0, blocks * n * r).reshape(blocks, n, r) * 0.05
     bias = normal(derive_seed("adaln-bias", seed, blocks, n), 0, blocks * n).reshape(blocks, n) * 0.01
     return to_bf16_bits(e), to_f16_bits(basis), to_f16_bits(proj), to_f16_bits(bias)
+
+
+# ---------------------------------------------------------------------------
+# The same recipes evaluated with torch on any device
+# ---------------------------------------------------------------------------
+#
+# Full-size workloads (the 168-layer block sweep draws ~50 G normals) are far
+# too large for numpy on the host, so the recipes are also written with torch
+# tensor operations that run where the tensors live.  The arithmetic is the
+# same step for step: SplitMix64 in uint64 arithmetic (held in int64 tensors;
+# multiplication wraps modulo 2^64, right shifts are made logical by masking),
+# the same uniform and Box-Muller formulas in binary64, and BF16
+# round-to-nearest-even straight from binary64.  The only possible difference
+# from the numpy path is the last-ulp rounding of log, cos and sin in the
+# device's libraries, which changes the BF16 result only when a draw lies
+# within ~1e-16 (relative) of a BF16 rounding boundary: about 1e-13 of draws.
+# Tests that consume these tensors always hand the oracle the very bytes the
+# GPU consumed, so parity never depends on the two paths agreeing.
+
+def _s64(v: int) -> int:
+    """uint64 value -> the int64 with the same bits."""
+    return v - (1 << 64) if v >= (1 << 63) else v
+
+
+_GAMMA_S = _s64(0x9E3779B97F4A7C15)
+_M1_S = _s64(0xBF58476D1CE4E5B9)
+_M2_S = _s64(0x94D049BB133111EB)
+
+
+def _srl(z, s: int):
+    """Logical right shift of int64 tensors holding uint64 bits."""
+    return (z >> s) & ((1 << (64 - s)) - 1)
+
+
+def _mix_t(z):
+    z = (z ^ _srl(z, 30)) * _M1_S
+    z = (z ^ _srl(z, 27)) * _M2_S
+    return z ^ _srl(z, 31)
+
+
+def u64_t(seed: int, start: int, n: int, device):
+    """Draws start .. start+n-1 of stream `seed` (int64 tensor of uint64 bits)."""
+    import torch
+    idx = torch.arange(start + 1, start + 1 + n, dtype=torch.int64, device=device)
+    return _mix_t(idx * _GAMMA_S + _s64(seed & 0xFFFFFFFFFFFFFFFF))
+
+
+def uniform_t(seed: int, start: int, n: int, device):
+    import torch
+    u = _srl(u64_t(seed, start, n, device), 11)
+    return (u.to(torch.float64) + 0.5) * (2.0 ** -53)
+
+
+def normal_t(seed: int, start: int, n: int, device):
+    """Standard normals start .. start+n-1 of stream `seed` (float64 tensor), as normal()."""
+    import torch
+    p0, p1 = start // 2, (start + n + 1) // 2
+    u = uniform_t(seed, 2 * p0, 2 * (p1 - p0), device).view(-1, 2)
+    r = torch.sqrt(-2.0 * torch.log(u[:, 0]))
+    t = (2.0 * np.pi) * u[:, 1]
+    z = torch.stack((r * torch.cos(t), r * torch.sin(t)), dim=1).view(-1)
+    off = start - 2 * p0
+    return z[off:off + n]
+
+
+def to_bf16_bits_t(x):
+    """Round a float64 tensor to BF16 (nearest, ties to even) directly from
+    binary64, as to_bf16_bits; returns int16 bits (view as torch.bfloat16)."""
+    import torch
+    m, e = torch.frexp(x)
+    r = torch.ldexp(torch.round(torch.ldexp(m, torch.full_like(e, 8))), e - 8)
+    return (r.to(torch.float32).view(torch.int32) >> 16).to(torch.int16)
+
+
+def truncated_normal_t(seed: int, start: int, n: int, device, bound: float = CLIP_LIMIT):
+    """truncated_normal() on `device`: draws at or beyond `bound` are redrawn
+    from the redraw sub-streams (rare: ~1e-15 of draws), on the host."""
+    import torch
+    z = normal_t(seed, start, n, device)
+    bad = torch.nonzero(z.abs() >= bound).view(-1)
+    if bad.numel():
+        idx = bad.cpu().numpy()
+        fix = np.empty(idx.size)
+        for j, i in enumerate(idx):
+            v, attempt = float(z[int(i)]), 0
+            while abs(v) >= bound:
+                attempt += 1
+                v = normal(derive_seed(seed, "redraw", attempt), start + int(i), 1)[0]
+            fix[j] = v
+        z[bad] = torch.from_numpy(fix).to(device)
+    return z
+
+
+def activation_batches_t(layer: Layer, b0: int, nb: int, device):
+    """activation_batches() on `device`: calibration-stream batches b0 ..
+    b0+nb-1 as int16 BF16 bits [nb * batch, K].  Recipes without injected
+    outliers only (the per-channel log-normal spread is supported)."""
+    import torch
+    if layer.outliers_per_batch():
+        raise ValueError("activation_batches_t: recipes with injected outliers run on the host")
+    B, K = layer.batch, layer.K
+    std = torch.from_numpy(channel_std(layer)).to(device) if layer.channel_lognormal else None
+    out = torch.empty((nb * B, K), dtype=torch.int16, device=device)
+    for j in range(nb):
+        z = truncated_normal_t(derive_seed(*layer.key, "x", b0 + j), 0, B * K, device)
+        if std is not None:
+            z = (z.view(B, K) * std[None, :]).view(-1)
+        out[j * B:(j + 1) * B] = to_bf16_bits_t(z).view(B, K)
+    return out
+
+
+def weights_t(layer: Layer, device):
+    """weights() on `device` as int16 BF16 bits [N, K]."""
+    return to_bf16_bits_t(normal_t(derive_seed(*layer.key, "w"), 0, layer.N * layer.K, device) * 0.02) \
+        .view(layer.N, layer.K)
+
+
+def bias_t(layer: Layer, device):
+    """bias() on `device` as int16 BF16 bits [N]."""
+    return to_bf16_bits_t(normal_t(derive_seed(*layer.key, "b"), 0, layer.N, device) * 0.01)

@@ -91,3 +91,30 @@ def test_adaln_inputs_shapes_and_spreads():
     np.testing.assert_array_equal(e2, e[[7, 0]])
     e0, *_ = S.adaln_inputs(1, 1, 64, 16, ())
     assert e0.shape == (0, 64)
+
+
+def test_torch_recipes_match_numpy_recipes_on_cpu():
+    """The torch restatement of the generator (used on the GPU for the full-size
+    workloads) gives the numpy recipe's BF16 bits: streams at odd offsets, the
+    log-normal channel spread, plain bodies, weights and biases."""
+    import torch
+    u = S.u64(12345678901234567890, 3, 7)
+    assert np.array_equal(u, S.u64_t(12345678901234567890, 3, 7, "cpu").numpy().view(np.uint64))
+    assert np.array_equal(S.normal(77, 5, 11), S.normal_t(77, 5, 11, "cpu").numpy())
+    sw = S.workloads()["block_sweep"]
+    for layer in (sw[0], sw[3]):                       # qkv-like (log-normal channels) and down (plain)
+        small = S.Layer(layer.name, 256, layer.K, 512, layer.batch, 8,
+                        channel_lognormal=layer.channel_lognormal, key=layer.key)
+        want = S.activation_batches(small, 2, 3)
+        got = S.activation_batches_t(small, 2, 3, "cpu").numpy().view(np.uint16)
+        assert np.array_equal(want, got)
+        assert np.array_equal(S.weights(small), S.weights_t(small, "cpu").numpy().view(np.uint16))
+        assert np.array_equal(S.bias(small), S.bias_t(small, "cpu").numpy().view(np.uint16))
+    x = np.array([1.0, -1.00390625, 1.001953125, 1.005859375, 3.0e38, -0.0, 65504.5, -7.99])
+    assert np.array_equal(S.to_bf16_bits(x), S.to_bf16_bits_t(torch.from_numpy(x)).numpy().view(np.uint16))
+
+
+def test_torch_recipes_refuse_outlier_recipes():
+    import pytest
+    with pytest.raises(ValueError):
+        S.activation_batches_t(S.workloads()["tiny"][0], 0, 1, "cpu")
