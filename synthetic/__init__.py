@@ -170,8 +170,10 @@ def channel_std(layer: Layer) -> np.ndarray:
     return np.exp(normal(derive_seed(*layer.key, "channel_std"), 0, layer.K))
 
 
-def activation_batches(layer: Layer, b0: int, nb: int, uncalibrated_body: bool = False) -> np.ndarray:
-    """Calibration-stream batches b0 .. b0+nb-1 of `layer` as BF16 bits [nb * batch, K]."""
+def activation_batches(layer: Layer, b0: int, nb: int, uncalibrated_body: bool = False,
+                       bound: float = CLIP_LIMIT) -> np.ndarray:
+    """Calibration-stream batches b0 .. b0+nb-1 of `layer` as BF16 bits [nb * batch, K]
+    (`bound`: the truncation of the body draws; the recipes use CLIP_LIMIT)."""
     B, K = layer.batch, layer.K
     out = np.empty((nb * B, K), dtype=np.uint16)
     std = channel_std(layer) if layer.channel_lognormal else None
@@ -179,7 +181,7 @@ def activation_batches(layer: Layer, b0: int, nb: int, uncalibrated_body: bool =
     for j in range(nb):
         b = b0 + j
         s = derive_seed(*layer.key, "x", b)
-        z = truncated_normal(s, 0, B * K)
+        z = truncated_normal(s, 0, B * K, bound)
         if std is not None:
             z = (z.reshape(B, K) * std[None, :]).reshape(-1)
         if n_out and not uncalibrated_body:
@@ -359,21 +361,43 @@ def truncated_normal_t(seed: int, start: int, n: int, device, bound: float = CLI
     return z
 
 
-def activation_batches_t(layer: Layer, b0: int, nb: int, device):
+def _normal_rows_t(seeds, n: int, device):
+    """Row j = normal(seeds[j], 0, n) for an even n, all rows at once ([len(seeds), n] float64)."""
+    import torch
+    sd = torch.tensor([_s64(v & 0xFFFFFFFFFFFFFFFF) for v in seeds], dtype=torch.int64, device=device)
+    idx = torch.arange(1, n + 1, dtype=torch.int64, device=device)
+    u = (_srl(_mix_t(idx[None, :] * _GAMMA_S + sd[:, None]), 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    u = u.view(len(seeds), n // 2, 2)
+    r = torch.sqrt(-2.0 * torch.log(u[:, :, 0]))
+    t = (2.0 * np.pi) * u[:, :, 1]
+    return torch.stack((r * torch.cos(t), r * torch.sin(t)), dim=2).view(len(seeds), n)
+
+
+def activation_batches_t(layer: Layer, b0: int, nb: int, device, chunk: int = 32, bound: float = CLIP_LIMIT):
     """activation_batches() on `device`: calibration-stream batches b0 ..
-    b0+nb-1 as int16 BF16 bits [nb * batch, K].  Recipes without injected
-    outliers only (the per-channel log-normal spread is supported)."""
+    b0+nb-1 as int16 BF16 bits [nb * batch, K], `chunk` batches per pass.
+    Recipes without injected outliers only (the per-channel log-normal spread
+    is supported)."""
     import torch
     if layer.outliers_per_batch():
         raise ValueError("activation_batches_t: recipes with injected outliers run on the host")
     B, K = layer.batch, layer.K
     std = torch.from_numpy(channel_std(layer)).to(device) if layer.channel_lognormal else None
     out = torch.empty((nb * B, K), dtype=torch.int16, device=device)
-    for j in range(nb):
-        z = truncated_normal_t(derive_seed(*layer.key, "x", b0 + j), 0, B * K, device)
+    for j0 in range(0, nb, chunk):
+        seeds = [derive_seed(*layer.key, "x", b0 + j) for j in range(j0, min(nb, j0 + chunk))]
+        z = _normal_rows_t(seeds, B * K, device)
+        bad = torch.nonzero(z.abs() >= bound)
+        for r, i in bad.cpu().tolist():             # truncation redraws: ~1e-15 of draws at bound 8
+            v, attempt = float(z[r, i]), 0
+            while abs(v) >= bound:
+                attempt += 1
+                v = normal(derive_seed(seeds[r], "redraw", attempt), i, 1)[0]
+            z[r, i] = v
+        z = z.view(len(seeds), B, K)
         if std is not None:
-            z = (z.view(B, K) * std[None, :]).view(-1)
-        out[j * B:(j + 1) * B] = to_bf16_bits_t(z).view(B, K)
+            z = z * std[None, None, :]
+        out[j0 * B:(j0 + len(seeds)) * B] = to_bf16_bits_t(z).view(len(seeds) * B, K)
     return out
 
 

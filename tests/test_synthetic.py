@@ -114,6 +114,17 @@ def test_torch_recipes_match_numpy_recipes_on_cpu():
     assert np.array_equal(S.to_bf16_bits(x), S.to_bf16_bits_t(torch.from_numpy(x)).numpy().view(np.uint16))
 
 
+def test_torch_recipes_redraw_like_numpy():
+    """With a truncation bound of 1.5 (a third of the draws redrawn, some more
+    than once) the torch path redraws exactly as the numpy path does."""
+    layer = S.workloads()["block_sweep"][3]
+    small = S.Layer(layer.name, 64, 64, 64, 8, 3, key=layer.key)
+    want = S.activation_batches(small, 0, 3, bound=1.5)
+    got = S.activation_batches_t(small, 0, 3, "cpu", chunk=2, bound=1.5).numpy().view(np.uint16)
+    assert np.array_equal(want, got)
+    assert (np.abs(S.bf16_to_f32(want)) <= 1.5).all()       # < 1.5 before the BF16 rounding
+
+
 def test_torch_recipes_refuse_outlier_recipes():
     import pytest
     with pytest.raises(ValueError):
