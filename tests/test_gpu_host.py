@@ -76,3 +76,23 @@ def test_back_to_back_calls_and_pageable_memory():
     for x_host, y_host in outs:
         y_ref, _ = _device_reference(x_host, wc, wsc, b)
         assert torch.equal(y_host.view(torch.int16), y_ref.view(torch.int16))
+
+
+def test_explicit_stream_with_owned_workspace():
+    """A call on a stream other than the current one, with the workspace left
+    to the binding: the workspace must stay reserved for that stream's work, so
+    allocations made on the current stream right after the call (which would
+    reuse a freed block) do not disturb the result."""
+    m = fh()
+    wc, wsc, b = _weights()
+    x_host = _x(9000, "side")
+    y_host = torch.empty((9000, N), dtype=torch.bfloat16).pin_memory()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    m.fh_nvfp4_linear_host(x_host, SG_A, wc, wsc, SG_W, b, y_host, None, chunk_rows=1024, stream=side)
+    junk = [torch.full((1 << 22,), 7, dtype=torch.int32, device="cuda") for _ in range(8)]
+    torch.cuda.synchronize()
+    m.fh_device_status()
+    del junk
+    y_ref, _ = _device_reference(x_host, wc, wsc, b)
+    assert torch.equal(y_host.view(torch.int16), y_ref.view(torch.int16))
