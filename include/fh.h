@@ -219,6 +219,42 @@ int fh_nvfp4_linear_host(const uint16_t* x_host, int64_t M, int64_t K, float a_g
  * shape is not supported. */
 size_t fh_nvfp4_linear_host_workspace_bytes(int64_t K, int64_t N, int64_t chunk_rows);
 
+/* Bytes of the library's static device scratch array (16 MiB). */
+#define FH_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* The layer on host buffers without any device allocation, for callers that
+ * cannot allocate device memory: a serving engine or host application that
+ * reserves the device's memory for its own pool up front, a plugin that may
+ * only use memory handed to it, or a caller that must not pay for cudaMalloc /
+ * cudaFree, which can synchronize the device.  The pages have no counterpart;
+ * this is a packaging of fh_nvfp4_linear_host.
+ * Computes the same y_host as fh_nvfp4_linear_host, byte for byte, but stages
+ * its row chunks in a scratch array that is part of the library's own device
+ * memory (FH_NOALLOC_SCRATCH_BYTES per device, held by every device on which
+ * the library's module is loaded until the process exits) instead of a
+ * caller's workspace.  The library calls no cudaMalloc or cudaFree here.
+ * Each chunk (the largest multiple of 128 rows whose x, codes, scales and
+ * output fit the array) is uploaded, quantized, multiplied and downloaded in
+ * order on `stream`; nothing overlaps inside a call.
+ * The first call on a device looks up the array's device address with that
+ * device current and keeps it; make that first call before any stream capture.
+ * Every call on a device shares the one array, and each call rewrites
+ * everything it reads from it, so the contents a previous call left are never
+ * used.  Calls whose work overlaps on the GPU (calls on two streams, or from
+ * two host threads, of one process) race on the array and corrupt each
+ * other's results: serialize them, for example on one stream.
+ * x_host, y_host, weights, bias and clip counter as for fh_nvfp4_linear_host.
+ * Requires K % 64 == 0, N % 8 == 0, and that one 128-row chunk fits the array:
+ * 128 * (2.5625 * K + 2 * N) bytes, plus alignment, at most
+ * FH_NOALLOC_SCRATCH_BYTES (FH_ERR_UNSUPPORTED_SHAPE otherwise, e.g.
+ * K = N = 2688 gives 1280-row chunks, K = 10752 with N = 2688 384-row ones).
+ * A CUDA error in the chunk loop returns FH_ERR_CUDA after part of the work was
+ * enqueued on `stream`; synchronize it before freeing the buffers. */
+int fh_nvfp4_linear_host_noalloc(const uint16_t* x_host, int64_t M, int64_t K, float a_gscale,
+                                 const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                                 const uint16_t* bias_dev, int64_t N, uint16_t* y_host,
+                                 unsigned long long* clip_count_dev, fh_stream_t stream);
+
 /* Permute FH_SCALES_MMA_TILED scales of a [rows, K] matrix into row-major
  * [rows, K/16] (drops the padding).  Requires K % 64 == 0. */
 int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows,

@@ -62,6 +62,8 @@ _SIG = {
     "fh_nvfp4_linear_host": (_c.c_int, [_P, _I64, _I64, _c.c_float, _P, _P, _c.c_float, _P, _I64, _P, _P, _I64, _P,
                                         _c.c_size_t, _P]),
     "fh_nvfp4_linear_host_workspace_bytes": (_c.c_size_t, [_I64, _I64, _I64]),
+    "fh_nvfp4_linear_host_noalloc": (_c.c_int, [_P, _I64, _I64, _c.c_float, _P, _P, _c.c_float, _P, _I64, _P, _P,
+                                                _P]),
     "fh_gelu_bf16": (_c.c_int, [_P, _P, _I64, _P]),
     "fh_quantize_int8_rows": (_c.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "fh_int8_attention_scores": (_c.c_int, [_P, _P, _P, _P, _c.c_float, _P, _I64, _I64, _I64, _I64, _P]),
@@ -275,6 +277,32 @@ def fh_nvfp4_linear_host(x_host: torch.Tensor, a_gscale: float, w_codes: torch.T
         # the caching allocator must not hand the block to other streams before
         # that work has finished.
         workspace.record_stream(torch_stream)
+
+
+def fh_nvfp4_linear_host_noalloc(x_host: torch.Tensor, a_gscale: float, w_codes: torch.Tensor,
+                                 w_scales: torch.Tensor, w_gscale: float, bias: torch.Tensor | None,
+                                 y_host: torch.Tensor, clip: torch.Tensor | None = None, stream=None) -> None:
+    """fh_nvfp4_linear_host without a workspace: the chunks are staged in the library's static device scratch
+    array (see include/fh.h), so nothing is allocated on the device.  Calls sharing a device must not overlap on
+    the GPU.  Ordered on the stream: synchronize before reading y_host."""
+    for t, n in ((x_host, "x_host"), (y_host, "y_host")):
+        if not isinstance(t, torch.Tensor) or t.device.type != "cpu" or t.dtype not in _BF16 or t.dim() != 2:
+            raise TypeError(f"{n} must be a 2-D BF16 CPU tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    _need(w_codes, _U8, "w_codes", 2)
+    _need(w_scales, _U8, "w_scales")
+    M, K = x_host.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K or tuple(y_host.shape) != (M, N):
+        raise ValueError("shape mismatch: x_host [M, K], w_codes [N, K/2], y_host [M, N]")
+    if bias is not None:
+        _need(bias, _BF16, "bias")
+    if clip is not None and (clip.dtype != torch.int64 or clip.device.type != "cuda"):
+        raise TypeError("clip must be a CUDA int64 tensor")
+    _check(_lib.fh_nvfp4_linear_host_noalloc(_P(x_host.data_ptr()), M, K, float(a_gscale), _ptr(w_codes),
+                                             _ptr(w_scales), float(w_gscale), _ptr(bias), N, _P(y_host.data_ptr()),
+                                             _ptr(clip), _stream(stream)))
 
 
 def fh_scales_to_rowmajor(tiled: torch.Tensor, rowmajor: torch.Tensor, rows: int, K: int, stream=None) -> None:

@@ -251,6 +251,37 @@ int fh_nvfp4_linear_host(const uint16_t* x_host, int64_t M, int64_t K, float a_g
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear_host");
 }
 
+int fh_nvfp4_linear_host_noalloc(const uint16_t* x_host, int64_t M, int64_t K, float a_gscale,
+                                 const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                                 const uint16_t* bias_dev, int64_t N, uint16_t* y_host,
+                                 unsigned long long* clip_count_dev, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!(a_gscale > 0.0f) || isinf(a_gscale) || !(w_gscale > 0.0f) || isinf(w_gscale))
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_host_noalloc: global scales must be finite and > 0%s");
+  if (M < 0 || M > 0x7FFFFFFF || K <= 0 || K % 64 != 0 || N <= 0 || N % 8 != 0 || K > 0x7FFFFFFF ||
+      N > 0x7FFFFFFF)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_nvfp4_linear_host_noalloc: need 0 <= M < 2^31, K > 0, K %% 64 == 0, N > 0, N %% 8 == 0%s");
+  if (fh::noalloc_chunk_rows(K, N) == 0) {
+    char msg[200];
+    snprintf(msg, sizeof msg, "one 128-row chunk needs %zu bytes of scratch, more than the library's static %u",
+             fh::noalloc_chunk_bytes(K, N, 128), (unsigned)FH_NOALLOC_SCRATCH_BYTES);
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_host_noalloc: %s", msg);
+  }
+  if (M == 0) return FH_OK;
+  if (x_host == nullptr || y_host == nullptr || w_codes_dev == nullptr || w_scales_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_host_noalloc: null pointer%s");
+  if (!aligned16(w_codes_dev) || !aligned16(w_scales_dev) || (bias_dev != nullptr && !aligned16(bias_dev)))
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_host_noalloc: weights and bias must be 16-byte aligned%s");
+  if (int st = check_device()) return st;
+  const char* why = nullptr;
+  cudaError_t e = fh::launch_nvfp4_linear_host_noalloc(x_host, M, K, a_gscale, w_codes_dev, w_scales_dev, w_gscale,
+                                                       bias_dev, N, y_host, clip_count_dev, (cudaStream_t)stream, &why);
+  if (e == cudaErrorNotSupported && why != nullptr)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_host_noalloc: %s", why);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear_host_noalloc");
+}
+
 int fh_scales_to_rowmajor(const uint8_t* tiled_dev, uint8_t* rowmajor_dev, int64_t rows, int64_t K,
                           fh_stream_t stream) {
   g_last_error[0] = 0;

@@ -124,4 +124,15 @@ cudaError_t launch_nvfp4_linear_host(const uint16_t* x_host, int64_t M, int64_t 
                                      uint16_t* y_host, unsigned long long* clip, int64_t chunk_rows, void* workspace,
                                      cudaStream_t s, const char** why);
 
+// The host-buffer layer staged in the library's static scratch array
+// (fh_noalloc.cu).  noalloc_chunk_rows: rows per chunk for K and N (a multiple
+// of 128), 0 if not even 128 rows fit; noalloc_chunk_bytes: scratch bytes one
+// chunk of that many rows uses.  Arguments are validated by the caller.
+int64_t noalloc_chunk_rows(int64_t K, int64_t N);
+size_t noalloc_chunk_bytes(int64_t K, int64_t N, int64_t rows);
+cudaError_t launch_nvfp4_linear_host_noalloc(const uint16_t* x_host, int64_t M, int64_t K, float a_g,
+                                             const uint8_t* w_codes, const uint8_t* w_scales, float w_g,
+                                             const uint16_t* bias, int64_t N, uint16_t* y_host,
+                                             unsigned long long* clip, cudaStream_t s, const char** why);
+
 }  // namespace fh
