@@ -375,13 +375,11 @@ def _normal_rows_t(seeds, n: int, device):
 
 def activation_batches_t(layer: Layer, b0: int, nb: int, device, chunk: int = 32, bound: float = CLIP_LIMIT):
     """activation_batches() on `device`: calibration-stream batches b0 ..
-    b0+nb-1 as int16 BF16 bits [nb * batch, K], `chunk` batches per pass.
-    Recipes without injected outliers only (the per-channel log-normal spread
-    is supported)."""
+    b0+nb-1 as int16 BF16 bits [nb * batch, K], `chunk` batches per pass
+    (every recipe: log-normal channel spreads and injected outliers)."""
     import torch
-    if layer.outliers_per_batch():
-        raise ValueError("activation_batches_t: recipes with injected outliers run on the host")
     B, K = layer.batch, layer.K
+    n_out = layer.outliers_per_batch()
     std = torch.from_numpy(channel_std(layer)).to(device) if layer.channel_lognormal else None
     out = torch.empty((nb * B, K), dtype=torch.int16, device=device)
     for j0 in range(0, nb, chunk):
@@ -394,11 +392,33 @@ def activation_batches_t(layer: Layer, b0: int, nb: int, device, chunk: int = 32
                 attempt += 1
                 v = normal(derive_seed(seeds[r], "redraw", attempt), i, 1)[0]
             z[r, i] = v
-        z = z.view(len(seeds), B, K)
         if std is not None:
-            z = z * std[None, None, :]
+            z = (z.view(len(seeds), B, K) * std[None, None, :]).view(len(seeds), B * K)
+        if n_out:
+            # The n_out positions with the lowest keys (keys compared as uint64:
+            # flipping the sign bit makes the int64 order the unsigned one).
+            keys = _normal_keys_t([derive_seed(s, "outlier_pos") for s in seeds], B * K, device)
+            pos = torch.topk(keys ^ _s64(1 << 63), n_out, dim=1, largest=False, sorted=True).indices
+            sign_u = torch.stack([uniform_t(derive_seed(s, "outlier_sign"), 0, n_out, device) for s in seeds])
+            sign = torch.where(sign_u < 0.5, -1.0, 1.0).to(torch.float64)
+            if layer.outlier_mode == "fixed":
+                mag = torch.full((len(seeds), n_out), OUTLIER_MAX_FACTOR * CLIP_LIMIT, dtype=torch.float64,
+                                 device=device)
+            else:
+                u = torch.stack([uniform_t(derive_seed(s, "outlier_mag"), 0, n_out, device) for s in seeds])
+                mag = CLIP_LIMIT * (1.0 + (OUTLIER_MAX_FACTOR - 1.0) * u)
+                mag[:, 0] = OUTLIER_MAX_FACTOR * CLIP_LIMIT
+            z.scatter_(1, pos, sign * mag)
         out[j0 * B:(j0 + len(seeds)) * B] = to_bf16_bits_t(z).view(len(seeds) * B, K)
     return out
+
+
+def _normal_keys_t(seeds, n: int, device):
+    """Row j = u64(seeds[j], 0, n) (int64 tensor of uint64 bits), all rows at once."""
+    import torch
+    sd = torch.tensor([_s64(v & 0xFFFFFFFFFFFFFFFF) for v in seeds], dtype=torch.int64, device=device)
+    idx = torch.arange(1, n + 1, dtype=torch.int64, device=device)
+    return _mix_t(idx[None, :] * _GAMMA_S + sd[:, None])
 
 
 def weights_t(layer: Layer, device):

@@ -125,7 +125,14 @@ def test_torch_recipes_redraw_like_numpy():
     assert (np.abs(S.bf16_to_f32(want)) <= 1.5).all()       # < 1.5 before the BF16 rounding
 
 
-def test_torch_recipes_refuse_outlier_recipes():
-    import pytest
-    with pytest.raises(ValueError):
-        S.activation_batches_t(S.workloads()["tiny"][0], 0, 1, "cpu")
+def test_torch_recipes_inject_outliers_like_numpy():
+    """Both outlier modes: fixed +-137 L (tiny workload) and L * U[1, 137] with
+    one exactly 137 L per batch (attention projection), at the same positions,
+    signs and magnitudes as the numpy recipe."""
+    tiny = S.workloads()["tiny"][0]
+    assert np.array_equal(S.activation_batches(tiny, 3, 2), S.activation_batches_t(tiny, 3, 2, "cpu").numpy().view(np.uint16))
+    ap = S.workloads()["attn_proj"][0]
+    small = S.Layer(ap.name, 128, 512, 64, ap.batch, 4, ap.outlier_rate * 8, ap.outlier_mode, key=ap.key)
+    assert small.outliers_per_batch() > 1
+    want = S.activation_batches(small, 1, 2)
+    assert np.array_equal(want, S.activation_batches_t(small, 1, 2, "cpu").numpy().view(np.uint16))
