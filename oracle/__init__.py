@@ -213,9 +213,12 @@ def gelu(x_bits: np.ndarray) -> np.ndarray:
 #   s = fp32(amax_row / 127)                      (IEEE single division)
 #   q = clamp(rne(fp32(x / s)), -127, 127)        (IEEE single division, then
 #                                                  round half to even)
-# with s = 0 and q = 0 for an all-zero row.  The decisions are taken in FP32
-# because the kernel takes them in FP32; numpy's float32 division is the IEEE
-# correctly rounded one.
+# with s = 0 and q = 0 for an all-zero row.  The decisions are taken in FP32:
+# the method keeps one scale per row and multiplies it back into the integer
+# scores, so that scale is a stored FP32 number, and the quotient that decides
+# each code is the quotient by that stored number, correctly rounded to FP32
+# like the scale itself (numpy's float32 division is the IEEE correctly
+# rounded one).
 
 def quantize_int8_rows(x_bits: np.ndarray):
     """BF16 bits [rows, d] -> (int8 [rows, d], float32 scales [rows])."""
@@ -240,8 +243,12 @@ def int8_scores(q8: np.ndarray, q_scales: np.ndarray, k8: np.ndarray, k_scales: 
 
 
 def int8_scores_tolerance(s_ref: np.ndarray) -> np.ndarray:
-    """Three FP32 roundings of an exact product: 2e-6 relative (2^-21 = 4.8e-7 each), plus 1e-30."""
-    return 2e-6 * np.abs(s_ref) + 1e-30
+    """Allowed |S - S_ref| for S = (float(acc) * (s_q * sm_scale)) * s_k evaluated in FP32: at
+    most four roundings separate it from the exact product (the conversion of acc, exact while
+    |acc| < 2^24, and the three multiplies), each within 2^-24 relative, so |S - S_ref| <=
+    ((1 + 2^-24)^4 - 1) |S_ref| < 4 * 2^-24 * (1 + 2^-20) |S_ref|; the factor also covers
+    the binary64 rounding of S_ref.  The 1e-30 absolute term covers FP32 underflow."""
+    return 4.0 * 2.0 ** -24 * (1.0 + 2.0 ** -20) * np.abs(s_ref) + 1e-30
 
 
 # ---- AdaLN timestep conditioning through a shared low-rank basis -------------------

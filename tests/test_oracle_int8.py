@@ -87,3 +87,28 @@ def test_int8_scores_dequantized_close_to_float_product():
     ref = S.bf16_to_f32(xq).astype(np.float64) @ S.bf16_to_f32(xk).astype(np.float64).T
     bound = 128 * (np.abs(S.bf16_to_f32(xq)).max() * ks.max() + np.abs(S.bf16_to_f32(xk)).max() * qs.max())
     assert np.abs(s - ref).max() <= bound
+
+
+def test_score_tolerance_covers_fp32_evaluation_and_no_more():
+    """The four-rounding bound: the scores evaluated in FP32 in the stated order
+    (float(acc) * (s_q * sm_scale)) * s_k -- here with numpy's float32, including
+    sums past 2^24 whose conversion rounds -- lie within the tolerance of the
+    binary64 scores, and values five FP32 ulps away do not."""
+    rng = np.random.default_rng(3)
+    d = 2688
+    q8 = rng.integers(-127, 128, size=(1, 24, d)).astype(np.int8)
+    q8[0, :4] = 127                                        # |acc| up to 127^2 d > 2^24: the conversion rounds
+    k8 = rng.integers(-127, 128, size=(1, 40, d)).astype(np.int8)
+    k8[0, :4] = 127
+    qs = rng.uniform(1e-3, 2.0, size=(1, 24)).astype(np.float32)
+    ks = rng.uniform(1e-3, 2.0, size=(1, 40)).astype(np.float32)
+    sm = np.float32(1.0 / np.sqrt(128.0))
+    ref = oracle.int8_scores(q8, qs, k8, ks, float(sm))
+    acc = np.einsum("hid,hjd->hij", q8.astype(np.int64), k8.astype(np.int64))
+    assert np.abs(acc).max() > 2 ** 24
+    s32 = (acc.astype(np.float32) * (qs * sm)[:, :, None]) * ks[:, None, :]
+    tol = oracle.int8_scores_tolerance(ref)
+    assert (np.abs(s32.astype(np.float64) - ref) <= tol).all()
+    far = ref * (1.0 + 5 * 2.0 ** -24) + np.sign(ref) * 1e-29
+    big = np.abs(ref) > 1e-20
+    assert (np.abs(far - ref)[big] > tol[big]).all()
