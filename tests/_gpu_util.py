@@ -85,3 +85,38 @@ def check_linear(y_dev: torch.Tensor, a_bits: np.ndarray, a_g: float, w_bits: np
     assert (err <= tol).all(), (f"{int((err > tol).sum())} of {err.size} outputs out of tolerance; worst at "
                                 f"{worst}: y={y[worst]}, ref={y_ref[worst]}, tol={tol[worst]}")
     return float((err / np.maximum(tol, 1e-300)).max())
+
+
+def tile_rows(M: int, salt: int = 0) -> np.ndarray:
+    """One row in every 128-row tile of an M-row output (its place inside the
+    tile moves from tile to tile, so every TMEM lane quadrant and both CTAs of
+    a 256-row pair tile are visited), plus the rows at the edges of the
+    matrix, of the 256-row pair tiles and of the 32-row quadrants."""
+    tiles = np.arange((M + 127) // 128)
+    rows = tiles * 128 + (tiles * 37 + salt * 11 + 5) % 128
+    edges = [0, 1, 31, 32, 63, 64, 95, 96, 127, 128, 255, 256, M - 257, M - 256, M - 129, M - 128, M - 2, M - 1]
+    rows = np.concatenate([rows, np.array(edges)])
+    return np.unique(rows[(rows >= 0) & (rows < M)]).astype(np.int64)
+
+
+def bits_of(t: torch.Tensor) -> np.ndarray:
+    """The uint16 BF16 bits of a CUDA bfloat16 (or int16) tensor, on the host."""
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def check_quantized(codes: torch.Tensor, scales: torch.Tensor, clip: int, x_bits: np.ndarray, sg: float):
+    """Bit-exact comparison of a tensor-core-layout quantization the GPU already
+    made (codes, scales, clip count) with the oracle's quantization of x_bits."""
+    M, K = x_bits.shape
+    oc, osc, ocl = oracle.quantize(x_bits, sg)
+    gc = codes.cpu().numpy()
+    bad = np.argwhere(gc != oc)
+    assert bad.size == 0, f"{len(bad)} code bytes differ, first at {bad[:5].tolist()}"
+    gs = scales.cpu().numpy()
+    off = oracle.tiled_scale_offsets(M, K)
+    np.testing.assert_array_equal(gs[off], osc)
+    rest = np.ones(gs.size, dtype=bool)
+    rest[off.reshape(-1)] = False
+    assert (gs[rest] == 0).all(), "padding scales must be zero"
+    assert clip == ocl
+    return ocl

@@ -8,12 +8,15 @@ import torch
 
 import oracle
 import synthetic as S
-from _gpu_util import check_linear, check_quantize, fh, quantize_tiled, sample_rows, to_dev
+from _gpu_util import (bits_of, check_linear, check_quantize, check_quantized, fh, quantize_tiled, sample_rows,
+                       tile_rows, to_dev)
 
 pytestmark = pytest.mark.gpu
 
 
-def run_layer(x_bits, w_bits, b_bits, sg_a, sg_w):
+def run_layer(x_bits, w_bits, b_bits, sg_a, sg_w, keep=None):
+    """Quantize x and W on the GPU and run the GEMM.  keep: a dict that receives
+    the GPU's activation codes, scales and clip count for a full comparison."""
     m = fh()
     M, K = x_bits.shape
     N = w_bits.shape[0]
@@ -24,6 +27,8 @@ def run_layer(x_bits, w_bits, b_bits, sg_a, sg_w):
     bias = None if b_bits is None else to_dev(b_bits)
     m.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, bias, y)
     torch.cuda.synchronize()
+    if keep is not None:
+        keep.update(codes=ac, scales=asc)
     return y, int(aclip.item())
 
 
@@ -77,38 +82,60 @@ def layer_case(name, idx=0, calib_batches=None):
 
 @pytest.mark.parametrize("name", ["attn_proj", "qkv"])
 def test_full_size_layer(name):
+    """Configs 2 and 3 at their stated sizes: the activation quantizer's whole
+    output (codes, scales, clip count) bit-exact against the oracle, the
+    weights' too, and the GEMM within tolerance on one row of every 128-row
+    tile (every column) plus the tile and matrix edges."""
     layer, x, w, b, sg_a, sg_w = layer_case(name)
-    y, clips = run_layer(x, w, b, sg_a, sg_w)
+    got = {}
+    y, clips = run_layer(x, w, b, sg_a, sg_w, keep=got)
     assert clips == 0
+    check_quantized(got["codes"], got["scales"], clips, x, sg_a)
     check_quantize(w, sg_w, 1)
-    rows = sample_rows(layer.M, 48)
-    check_linear(y, x, sg_a, w, sg_w, b, rows=rows)
+    check_linear(y, x, sg_a, w, sg_w, b, rows=tile_rows(layer.M))
     assert not torch.isnan(y).any()
 
 
 def test_ffn_pair_with_gelu():
-    """Up-projection, GELU on BF16, re-quantization with the down layer's own
-    calibrated scale, down-projection; both quantizers clip nothing."""
+    """Config 4 at its stated size: up-projection 32768 x 2688 -> 10752, GELU on
+    BF16, the down layer's calibration over the GELU outputs of the same batches
+    (reading R10), its quantizer's whole 32768 x 10752 output bit-exact against
+    the oracle, and the down-projection.  Both quantizers clip nothing; both
+    GEMMs are checked on one row of every 128-row tile plus the edges.  (The up
+    layer's inputs carry one outlier of exactly 137 L in every batch, so its
+    amax over the evaluation batches equals the amax over all 1000.)"""
     m = fh()
     up = S.workloads()["ffn"][0]
     down = S.workloads()["ffn"][1]
     _, x, w1, b1, sg_x, sg_w1 = layer_case("ffn", 0, calib_batches=up.n_eval_batches)
     w2, b2 = S.weights(down), S.bias(down)
     sg_w2 = oracle.scale_from_amax(oracle.amax(w2))
-    h, clips = run_layer(x, w1, b1, sg_x, sg_w1)
+    got = {}
+    h, clips = run_layer(x, w1, b1, sg_x, sg_w1, keep=got)
     assert clips == 0
+    check_quantized(got["codes"], got["scales"], clips, x, sg_x)
+    check_linear(h, x, sg_x, w1, sg_w1, b1, rows=tile_rows(up.M, salt=1))
+    del got
     g = torch.empty_like(h)
     m.fh_gelu_bf16(h, g)
+    del h
     amax = torch.zeros(1, dtype=torch.float32, device="cuda")
     m.fh_amax(g, amax)                         # the down layer's calibration over the same batches
     torch.cuda.synchronize()
+    g_bits = bits_of(g)
+    assert amax.item() == oracle.amax(g_bits)
     sg_h = m.fh_scale_from_amax(amax.item())
-    g_bits = g.view(torch.int16).cpu().numpy().view(np.uint16)
-    rows = sample_rows(up.M, 32, seed=3)
-    check_quantize(g_bits[rows], sg_h, 1)
-    y, clips2 = run_layer(g_bits, w2, b2, sg_h, sg_w2)
-    assert clips2 == 0
-    check_linear(y, g_bits, sg_h, w2, sg_w2, b2, rows=rows)
+    assert sg_h == oracle.scale_from_amax(amax.item())
+    gc, gsc, gclip = quantize_tiled(g, sg_h)   # the 32768 x 10752 launch that feeds the down GEMM
+    wc, wsc, _ = quantize_tiled(to_dev(w2), sg_w2)
+    y = torch.full((up.M, down.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    m.fh_nvfp4_linear(gc, gsc, sg_h, wc, wsc, sg_w2, to_dev(b2), y)
+    torch.cuda.synchronize()
+    assert int(gclip.item()) == 0
+    check_quantized(gc, gsc, 0, g_bits, sg_h)
+    check_quantize(w2, sg_w2, 1)
+    check_linear(y, g_bits, sg_h, w2, sg_w2, b2, rows=tile_rows(up.M, salt=2))
+    assert not torch.isnan(y).any()
 
 
 def test_block_sweep_layers_sampled():
@@ -253,3 +280,22 @@ def test_gemm_stall_times_out_drains_and_context_survives(monkeypatch):
     rows = sample_rows(1024, 64, seed=5)
     check_linear(y, x, sg_a, w, sg_w, None, rows=rows)
     m.fh_device_status()
+
+
+def test_mma_rate_probe_runs_and_stays_below_the_clock_table_peak():
+    """The FP4 tensor-rate probe (a measurement aid) runs with and without the
+    scale copies, leaves no error behind, and its rate stays below what the
+    clock table allows (148 SMs x 16384 FP4 MACs per cycle at 1965 MHz)."""
+    m = fh()
+    m.fh_device_status()
+    for copies in (False, True):
+        m.fh_selftest_mma_rate(1000, copies)                  # warm-up
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pairs = m.fh_selftest_mma_rate(20000, copies)
+        e1.record()
+        torch.cuda.synchronize()
+        m.fh_device_status()
+        assert 1 <= pairs <= torch.cuda.get_device_properties(0).multi_processor_count // 2
+        rate = pairs * 20000 * 2.0 * 256 * 256 * 256 / (e0.elapsed_time(e1) * 1e-3)
+        assert 1e15 < rate < 148 * 16384 * 2 * 1.965e9 * 1.02, rate
