@@ -24,9 +24,13 @@ namespace fh {
 
 struct __align__(16) QuantTable {
   uint16_t code_thr[128][8];  // [c][j<7]: smallest |x| (BF16 bits) whose exact magnitude code is >= j+1 at scale code c
-  uint16_t scale_thr[128];    // [c]: smallest block amax (BF16 bits) whose exact scale code is >= c
-  float inv[128];             // 1 / (S_c * s_g): multiplier of the converter path (0 for c == 0)
-  uint32_t fast_ok[4];        // bit c: the converter path is exact at scale code c
+  // Per scale code c, everything one block needs in one 8-byte load:
+  //   x: the FP32 bits of 1 / (S_c * s_g), the multiplier of the converter path
+  //      (0 for c == 0);
+  //   y: bits 0..14 the smallest block amax (BF16 magnitude bits) whose exact
+  //      scale code is >= c, bit 15 set when the converter path is exact at c,
+  //      bits 16..30 the same threshold for code c + 1 (+Inf bits for c = 126).
+  uint2 sc[128];
 };
 static_assert(sizeof(QuantTable) % 16 == 0, "table copy granularity");
 
@@ -104,13 +108,18 @@ __device__ __forceinline__ uint32_t quantize_block_codes(const QuantTable& tab, 
   const uint32_t r45 = max_abs_bf16x2(w[4], w[5]), r67 = max_abs_bf16x2(w[6], w[7]);
   const uint32_t r = max_abs_bf16x2(max_abs_bf16x2(r01, r23), max_abs_bf16x2(r45, r67));
   const uint32_t amax = max_abs_bf16x2(r, __byte_perm(r, 0, 0x1032)) & 0x7FFFu;
-  // Scale code: converter candidate, corrected against the exact thresholds.
+  // Scale code: converter candidate, corrected against the exact thresholds
+  // (the candidate is almost always right: one table load checks it).
   const float amax_f = bf16_to_float(amax);
   uint32_t c = min(cvt_e4m3_sat(amax_f * inv6sg), 126u);
-  while (c < 126u && amax >= tab.scale_thr[c + 1]) ++c;
-  while (c > 0u && amax < tab.scale_thr[c]) --c;
-  const float inv = tab.inv[c];
-  if (((tab.fast_ok[c >> 5] >> (c & 31)) & 1u) && (amax_f * inv <= 3.0e38f)) {
+  uint2 e = tab.sc[c];
+  if (amax < (e.y & 0x7FFFu) || amax >= (e.y >> 16)) {
+    while (c < 126u && amax >= (tab.sc[c].y >> 16)) ++c;
+    while (c > 0u && amax < (tab.sc[c].y & 0x7FFFu)) --c;
+    e = tab.sc[c];
+  }
+  const float inv = __uint_as_float(e.x);
+  if (((e.y >> 15) & 1u) && (amax_f * inv <= 3.0e38f)) {
     codes = make_uint2(cvt_e2m1x8(inv, w[0], w[1], w[2], w[3]), cvt_e2m1x8(inv, w[4], w[5], w[6], w[7]));
   } else {
     codes = codes_exact(tab, c, make_uint4(w[0], w[1], w[2], w[3]), make_uint4(w[4], w[5], w[6], w[7]));

@@ -115,16 +115,19 @@ void build_table(float sg_f, QuantTable* t) {
   const double sg = (double)sg_f;
   static const double e2m1_mid[7] = {0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0};
   memset(t, 0, sizeof *t);
+  uint16_t scale_thr[128];  // [c]: smallest block amax (BF16 bits) whose exact scale code is >= c
+  float inv[128];           // 1 / (S_c * s_g): multiplier of the converter path (0 for c == 0)
+  bool fast_ok[128] = {};   // the converter path is exact at scale code c
   for (int c = 0; c < 128; ++c) {
     // Block scale: codes c-1 and c meet at their midpoint; a tie goes to the even code.
     if (c == 0) {
-      t->scale_thr[c] = 0;
+      scale_thr[c] = 0;
     } else if (c == 127) {
-      t->scale_thr[c] = (uint16_t)kBf16Inf;  // NaN code: never chosen
+      scale_thr[c] = (uint16_t)kBf16Inf;  // NaN code: never chosen
     } else {
       const double lo = (c == 1) ? 0.0 : e4m3_magnitude(c - 1);
       const double mid = 0.5 * (lo + e4m3_magnitude(c));
-      t->scale_thr[c] = (uint16_t)bf16_threshold(mid * 6.0 * sg, ((c - 1) & 1) == 0);
+      scale_thr[c] = (uint16_t)bf16_threshold(mid * 6.0 * sg, ((c - 1) & 1) == 0);
     }
     // Element codes at scale code c: magnitude codes j and j+1 meet at the grid
     // midpoint times S_c * s_g; a tie goes to the even code.
@@ -134,7 +137,7 @@ void build_table(float sg_f, QuantTable* t) {
         v = bf16_threshold(e2m1_mid[j] * e4m3_magnitude(c) * sg, (j & 1) == 0);
       t->code_thr[c][j] = (uint16_t)v;
     }
-    t->inv[c] = (c == 0 || c == 127) ? 0.0f : (float)(1.0 / (e4m3_magnitude(c) * sg));
+    inv[c] = (c == 0 || c == 127) ? 0.0f : (float)(1.0 / (e4m3_magnitude(c) * sg));
   }
   // Converter path check at both sides of every boundary and at the ends of the
   // BF16 range.  Negative inputs give the same magnitude with the sign bit set.
@@ -165,16 +168,23 @@ void build_table(float sg_f, QuantTable* t) {
       }
       return ok;
     };
-    const float inv0 = t->inv[c];
+    const float inv0 = inv[c];
     const float up1 = nextafterf(inv0, INFINITY), dn1 = nextafterf(inv0, 0.0f);
     const float cand[5] = {inv0, up1, dn1, nextafterf(up1, INFINITY), nextafterf(dn1, 0.0f)};
-    for (float inv : cand) {
-      if (passes(inv)) {
-        t->inv[c] = inv;
-        t->fast_ok[c >> 5] |= 1u << (c & 31);
+    for (float m : cand) {
+      if (passes(m)) {
+        inv[c] = m;
+        fast_ok[c] = true;
         break;
       }
     }
+  }
+  // The packed per-code entries the kernels read.
+  for (int c = 0; c < 128; ++c) {
+    uint32_t bits;
+    memcpy(&bits, &inv[c], 4);
+    const uint32_t next = (c < 127) ? scale_thr[c + 1] : kBf16Inf;
+    t->sc[c] = make_uint2(bits, (uint32_t)scale_thr[c] | (fast_ok[c] ? 0x8000u : 0u) | (next << 16));
   }
 }
 
