@@ -154,11 +154,49 @@ int fh_gelu_quantize_act(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ld
  * of the default 256 x 256 (both give identical results);
  * FH_GEMM_TEST_STALL=1 (read at each launch) is a test hook that makes the
  * first CTA group's MMA warp stop after three stages of its first tile
- * (K >= 1024), so the call ends with FH_ERR_TIMEOUT. */
+ * (K >= 1024), and FH_GEMM_TEST_STALL=2 one that makes the second CTA of the
+ * first pair stop loading after two stages; either call ends with
+ * FH_ERR_TIMEOUT after draining what it issued. */
 int fh_nvfp4_linear(const uint8_t* a_codes_dev, const uint8_t* a_scales_dev, float a_gscale,
                     const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
                     const uint16_t* bias_dev, uint16_t* y_dev, int64_t M, int64_t N,
                     int64_t K, fh_stream_t stream);
+
+/* The NVFP4 linear layer with the quantization of its BF16 input fused into
+ * the same kernel (FastH3 Trim, "How fast it runs": the FP8 path's fused
+ * per-tensor kernel; FastH3 thread digest, tweet 6/8: every FP4 layer's input
+ * quantized with its calibrated scale).  Computes exactly fh_quantize_act
+ * (FH_SCALES_MMA_TILED) followed by fh_nvfp4_linear, with byte-identical
+ * results, in one launch: two warps of every CTA quantize x while the tensor
+ * cores multiply the row blocks already quantized, so the quantization runs
+ * under the GEMM instead of before it.
+ *   x          BF16 [M, K], rows ldx elements apart (ldx >= K, ldx % 8 == 0)
+ *   a_codes, a_scales  outputs: x's codes [M, K/2] and tensor-core-layout
+ *              scales (fh_scales_bytes(M, K, FH_SCALES_MMA_TILED) bytes), as
+ *              fh_quantize_act writes them; the GEMM reads them back from L2
+ *   clip_count device counter, incremented as by fh_quantize_act (may be NULL)
+ *   sync       fh_nvfp4_linear_fused_quant_sync_bytes(M) bytes of device
+ *              scratch the caller owns: ceil(M/128) row-block ready counters
+ *              and an exit counter.  It must be zero before the first call
+ *              (e.g. cudaMemsetAsync); every call leaves it zero again,
+ *              including a call that ends with FH_ERR_TIMEOUT.  Calls that
+ *              overlap on the GPU must use different sync buffers.
+ *   w_codes, w_scales, bias, y, N  as for fh_nvfp4_linear.
+ * Requires K % 64 == 0, N % 8 == 0, 16-byte aligned pointers (sync 4-byte).
+ * The kernel's CTAs wait on one another (a row block is quantized by other
+ * CTAs than the ones that multiply it), so the grid is sized to the CTA pairs
+ * that fit on the device at once; if other work keeps SMs busy for seconds,
+ * the bounded waits expire and the call reports FH_ERR_TIMEOUT through
+ * fh_device_status instead of hanging. */
+int fh_nvfp4_linear_fused_quant(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx, float a_gscale,
+                                const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                                const uint16_t* bias_dev, uint16_t* y_dev, int64_t N, uint8_t* a_codes_dev,
+                                uint8_t* a_scales_dev, unsigned long long* clip_count_dev, uint32_t* sync_dev,
+                                fh_stream_t stream);
+
+/* Bytes of the sync scratch fh_nvfp4_linear_fused_quant needs for M rows
+ * (0 for M < 0 or M >= 2^31). */
+size_t fh_nvfp4_linear_fused_quant_sync_bytes(int64_t M);
 
 /* The NVFP4 linear layer fused with the activation that follows it and with
  * the quantization of the next layer's input: the FFN's up projection, whose
@@ -329,6 +367,18 @@ int fh_adaln_modulation(const uint16_t* temb_dev, int64_t bt, int64_t d, const u
  * failure handling; this exists so the timeout path can be tested without
  * hanging or faulting a GPU. */
 int fh_selftest_bounded_wait(uint32_t limit_us, fh_stream_t stream);
+
+/* Measurement of the FP4 tensor rate, not part of the layer (the pages give no
+ * kernel-level figures): enqueues one CTA pair per pair of SMs, each issuing
+ * `iters` rounds of four tcgen05.mma cta_group::2 kind::mxf4nvf4 block_scale
+ * instructions of 256 x 256 x 64 -- the instruction and tile of
+ * fh_nvfp4_linear -- on operands resident in shared memory, so no global
+ * memory is touched.  with_scale_copies != 0 precedes every round with the
+ * twelve tcgen05.cp scale-atom copies the GEMM issues per 256-deep K stage.
+ * Each round is 2 * 256 * 256 * 256 FLOP per pair; time the call with events
+ * on `stream`.  *pairs_out (host) receives the number of pairs launched.
+ * 1 <= iters <= 1e6 (about 0.3 s at most). */
+int fh_selftest_mma_rate(int32_t iters, int32_t with_scale_copies, int32_t* pairs_out, fh_stream_t stream);
 
 /* Synchronizes `stream`, then reads and clears the device error word of the
  * current device.  Returns FH_OK, FH_ERR_TIMEOUT if a kernel gave up on a

@@ -59,6 +59,9 @@ _SIG = {
     "fh_nvfp4_linear_gelu_quant": (_c.c_int, [_P, _P, _c.c_float, _P, _P, _c.c_float, _P, _c.c_float, _P, _P, _P,
                                               _I64, _I64, _I64, _P]),
     "fh_scales_to_rowmajor": (_c.c_int, [_P, _P, _I64, _I64, _P]),
+    "fh_nvfp4_linear_fused_quant": (_c.c_int, [_P, _I64, _I64, _I64, _c.c_float, _P, _P, _c.c_float, _P, _P, _I64,
+                                               _P, _P, _P, _P, _P]),
+    "fh_nvfp4_linear_fused_quant_sync_bytes": (_c.c_size_t, [_I64]),
     "fh_nvfp4_linear_host": (_c.c_int, [_P, _I64, _I64, _c.c_float, _P, _P, _c.c_float, _P, _I64, _P, _P, _I64, _P,
                                         _c.c_size_t, _P]),
     "fh_nvfp4_linear_host_workspace_bytes": (_c.c_size_t, [_I64, _I64, _I64]),
@@ -69,6 +72,7 @@ _SIG = {
     "fh_int8_attention_scores": (_c.c_int, [_P, _P, _P, _P, _c.c_float, _P, _I64, _I64, _I64, _I64, _P]),
     "fh_adaln_modulation": (_c.c_int, [_P, _I64, _I64, _P, _I64, _P, _P, _I64, _I64, _P, _P, _P]),
     "fh_device_status": (_c.c_int, [_P]),
+    "fh_selftest_mma_rate": (_c.c_int, [_c.c_int32, _c.c_int32, _c.POINTER(_c.c_int32), _P]),
     "fh_selftest_bounded_wait": (_c.c_int, [_c.c_uint32, _P]),
 }
 for _name, (_res, _args) in _SIG.items():
@@ -236,6 +240,47 @@ def fh_nvfp4_linear_gelu_quant(a_codes: torch.Tensor, a_scales: torch.Tensor, a_
                                            _stream(stream)))
 
 
+def fh_nvfp4_linear_fused_quant_sync_bytes(M: int) -> int:
+    return _lib.fh_nvfp4_linear_fused_quant_sync_bytes(M)
+
+
+def empty_fused_sync(M: int, device="cuda") -> torch.Tensor:
+    """A zeroed sync buffer for fh_nvfp4_linear_fused_quant (each call leaves it zero again)."""
+    return torch.zeros(max(1, fh_nvfp4_linear_fused_quant_sync_bytes(M) // 4), dtype=torch.int32, device=device)
+
+
+def fh_nvfp4_linear_fused_quant(x: torch.Tensor, a_gscale: float, w_codes: torch.Tensor, w_scales: torch.Tensor,
+                                w_gscale: float, bias: torch.Tensor | None, y: torch.Tensor, a_codes: torch.Tensor,
+                                a_scales: torch.Tensor, clip: torch.Tensor | None, sync: torch.Tensor,
+                                stream=None) -> None:
+    """y [M, N] = the NVFP4 layer on BF16 x [M, K] with the quantization in the same kernel; also writes x's
+    codes and tensor-core-layout scales into a_codes / a_scales (see include/fh.h).  sync: empty_fused_sync(M)."""
+    _need(x, _BF16, "x", 2)
+    _need(w_codes, _U8, "w_codes", 2)
+    _need(w_scales, _U8, "w_scales")
+    _need(y, _BF16, "y", 2)
+    _need(a_codes, _U8, "a_codes", 2)
+    _need(a_scales, _U8, "a_scales")
+    _need(sync, (torch.int32, torch.uint32), "sync")
+    if x.stride(1) != 1 or not (y.is_contiguous() and a_codes.is_contiguous() and w_codes.is_contiguous()):
+        raise ValueError("x rows must be contiguous; y, a_codes, w_codes contiguous")
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K or tuple(y.shape) != (M, N) or tuple(a_codes.shape) != (M, K // 2):
+        raise ValueError("shape mismatch: x [M, K], w_codes [N, K/2], y [M, N], a_codes [M, K/2]")
+    if a_scales.numel() < fh_scales_bytes(M, K, FH_SCALES_MMA_TILED):
+        raise ValueError("a_scales too small")
+    if sync.numel() * 4 < fh_nvfp4_linear_fused_quant_sync_bytes(M):
+        raise ValueError("sync too small")
+    if bias is not None:
+        _need(bias, _BF16, "bias")
+    if clip is not None and (clip.dtype != torch.int64 or clip.device.type != "cuda"):
+        raise TypeError("clip must be a CUDA int64 tensor")
+    _check(_lib.fh_nvfp4_linear_fused_quant(_ptr(x), M, K, x.stride(0), float(a_gscale), _ptr(w_codes),
+                                            _ptr(w_scales), float(w_gscale), _ptr(bias), _ptr(y), N, _ptr(a_codes),
+                                            _ptr(a_scales), _ptr(clip), _ptr(sync), _stream(stream)))
+
+
 def fh_nvfp4_linear_host_workspace_bytes(K: int, N: int, chunk_rows: int = 4096) -> int:
     return _lib.fh_nvfp4_linear_host_workspace_bytes(K, N, chunk_rows)
 
@@ -382,6 +427,14 @@ def fh_adaln_modulation(temb: torch.Tensor, basis: torch.Tensor, proj: torch.Ten
 def fh_selftest_bounded_wait(limit_us: int, stream=None) -> None:
     """Enqueue the bounded-wait self-test (see include/fh.h); fh_device_status then reports the timeout."""
     _check(_lib.fh_selftest_bounded_wait(int(limit_us), _stream(stream)))
+
+
+def fh_selftest_mma_rate(iters: int, with_scale_copies: bool = False, stream=None) -> int:
+    """Enqueue the FP4 tensor-rate probe (see include/fh.h); returns the number of CTA pairs.
+    Each pair performs iters * 2 * 256 * 256 * 256 FLOP."""
+    pairs = _c.c_int32(0)
+    _check(_lib.fh_selftest_mma_rate(int(iters), 1 if with_scale_copies else 0, _c.byref(pairs), _stream(stream)))
+    return pairs.value
 
 
 def fh_device_status(stream=None) -> None:

@@ -209,6 +209,44 @@ int fh_nvfp4_linear_gelu_quant(const uint8_t* a_codes_dev, const uint8_t* a_scal
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear_gelu_quant launch");
 }
 
+size_t fh_nvfp4_linear_fused_quant_sync_bytes(int64_t M) {
+  if (M < 0 || M > 0x7FFFFFFF) return 0;
+  return (size_t)((M + 127) / 128 + 1) * sizeof(uint32_t);
+}
+
+int fh_nvfp4_linear_fused_quant(const uint16_t* x_dev, int64_t M, int64_t K, int64_t ldx, float a_gscale,
+                                const uint8_t* w_codes_dev, const uint8_t* w_scales_dev, float w_gscale,
+                                const uint16_t* bias_dev, uint16_t* y_dev, int64_t N, uint8_t* a_codes_dev,
+                                uint8_t* a_scales_dev, unsigned long long* clip_count_dev, uint32_t* sync_dev,
+                                fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (!(a_gscale > 0.0f) || isinf(a_gscale) || !(w_gscale > 0.0f) || isinf(w_gscale))
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_fused_quant: global scales must be finite and > 0%s");
+  if (M < 0 || N < 0 || K <= 0 || K % 64 != 0 || N % 8 != 0 || ldx < K || ldx % 8 != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_nvfp4_linear_fused_quant: need M, N >= 0, K > 0, K %% 64 == 0, N %% 8 == 0, ldx >= K, "
+                "ldx %% 8 == 0%s");
+  if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF || ((M + 127) / 128) * (K / 16) > 0x7FFFFFFF)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_fused_quant: tensor too large%s");
+  if (M == 0 || N == 0) return FH_OK;
+  if (x_dev == nullptr || w_codes_dev == nullptr || w_scales_dev == nullptr || y_dev == nullptr ||
+      a_codes_dev == nullptr || a_scales_dev == nullptr || sync_dev == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_nvfp4_linear_fused_quant: null pointer%s");
+  if (!aligned16(x_dev) || !aligned16(w_codes_dev) || !aligned16(w_scales_dev) || !aligned16(y_dev) ||
+      !aligned16(a_codes_dev) || !aligned16(a_scales_dev) || (bias_dev != nullptr && !aligned16(bias_dev)) ||
+      (reinterpret_cast<uintptr_t>(sync_dev) & 3u) != 0)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE,
+                "fh_nvfp4_linear_fused_quant: sync must be 4-byte aligned, every other pointer 16-byte aligned%s");
+  if (int st = check_device()) return st;
+  const char* why = nullptr;
+  cudaError_t e = fh::launch_nvfp4_linear_quant_prologue(x_dev, ldx, a_gscale, w_codes_dev, w_scales_dev, w_gscale,
+                                                         bias_dev, y_dev, a_codes_dev, a_scales_dev, clip_count_dev,
+                                                         sync_dev, M, N, K, (cudaStream_t)stream, &why);
+  if (e == cudaErrorNotSupported && why != nullptr)
+    return fail(FH_ERR_UNSUPPORTED_SHAPE, "fh_nvfp4_linear_fused_quant: %s", why);
+  return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_nvfp4_linear_fused_quant launch");
+}
+
 size_t fh_nvfp4_linear_host_workspace_bytes(int64_t K, int64_t N, int64_t chunk_rows) {
   if (K <= 0 || K % 64 != 0 || N <= 0 || N % 8 != 0 || chunk_rows <= 0 || chunk_rows % 128 != 0 ||
       K > 0x7FFFFFFF || N > 0x7FFFFFFF || chunk_rows > 0x7FFFFFFF)
@@ -386,6 +424,18 @@ int fh_selftest_bounded_wait(uint32_t limit_us, fh_stream_t stream) {
   if (int st = check_device()) return st;
   cudaError_t e = fh::launch_bounded_wait_selftest((uint64_t)limit_us * 1000u, (cudaStream_t)stream);
   return e == cudaSuccess ? FH_OK : cuda_fail(e, "fh_selftest_bounded_wait launch");
+}
+
+int fh_selftest_mma_rate(int32_t iters, int32_t with_scale_copies, int32_t* pairs_out, fh_stream_t stream) {
+  g_last_error[0] = 0;
+  if (iters < 1 || iters > 1000000 || pairs_out == nullptr)
+    return fail(FH_ERR_INVALID_ARG, "fh_selftest_mma_rate: need 1 <= iters <= 1e6 and pairs_out%s");
+  if (int st = check_device()) return st;
+  int pairs = 0;
+  cudaError_t e = fh::launch_mma_rate_probe((int)iters, with_scale_copies ? 1 : 0, &pairs, (cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "fh_selftest_mma_rate launch");
+  *pairs_out = pairs;
+  return FH_OK;
 }
 
 int fh_device_status(fh_stream_t stream) {

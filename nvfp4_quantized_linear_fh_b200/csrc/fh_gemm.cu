@@ -84,18 +84,24 @@ constexpr int kSfBufs = 2;
 // -- drained into registers by eight epilogue warps (two per TMEM lane
 // quadrant, one per 128-column half), which release it before they scale,
 // round and store; each stage then feeds 33% more MACs from 12% more bytes.
-template <int kCta, int kBN>
+// kPro = 1 (256-wide pair form only): the activations arrive in BF16 and two
+// more warps per CTA quantize them inside the kernel (see the prologue
+// quantizer below); one stage fewer makes room for their decision table.
+template <int kCta, int kBN, int kPro = 0>
 struct Cfg {
   static_assert(kBN == 192 || (kBN == 256 && kCta == 2), "tile forms");
+  static_assert(kPro == 0 || (kBN == 256 && kCta == 2), "the quantizing prologue runs in the 256-wide pair form");
   static constexpr int BN = kBN;                       // output columns per tile
   static constexpr int BM = 128 * kCta;                // output rows per tile
   static constexpr int kBRows = BN / kCta;             // W rows each CTA loads
   static constexpr int kAccBufs = BN == 256 ? 1 : 2;   // TMEM accumulators
   static constexpr int kEpiWarps = BN == 256 ? 8 : 4;
   static constexpr int kWarpCols = BN == 256 ? 128 : BN;  // accumulator columns per epilogue warp
-  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  static constexpr int kQuantWarps = kPro ? 2 : 0;     // prologue quantizer warps (warps 2, 3)
+  static constexpr int kEpiWarp0 = 2 + kQuantWarps;    // first epilogue warp
+  static constexpr int kThreads = 64 + 32 * kQuantWarps + 32 * kEpiWarps;
   static constexpr int kSfCol0 = kAccBufs * BN;        // first TMEM column of the scale buffers
-  static constexpr int kStages = BN == 256 ? 5 : (kCta == 2 ? 6 : 4);
+  static constexpr int kStages = BN == 256 ? (kPro ? 4 : 5) : (kCta == 2 ? 6 : 4);
   static constexpr int kEpiBufs = kCta == 2 ? 1 : 2;   // output staging buffers per epilogue warp
   static constexpr int kBBytes = kBRows * BK / 2;
   static constexpr int kOffA = 0;
@@ -104,9 +110,11 @@ struct Cfg {
   static constexpr int kOffSFB = kOffSFA + kStages * kSFABytes;
   static constexpr int kOffEpi = kOffSFB + kStages * kSFBBytes;
   static constexpr int kOffBias = kOffEpi + kEpiWarps * kEpiBufs * kEpiBufBytes;
-  static constexpr int kOffBar = kOffBias + kEpiWarps * kWarpCols * 2;
-  // full, empty (per stage); acc full, acc empty (per accumulator); drain
-  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 1;
+  static constexpr int kOffQTab = kOffBias + kEpiWarps * kWarpCols * 2;  // prologue decision table
+  static constexpr int kOffBar = kOffQTab + (kPro ? (int)sizeof(QuantTable) : 0);
+  // full, empty (per stage); acc full, acc empty (per accumulator); drain;
+  // the peer producer's end-of-loading report (leader CTA)
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 2;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
   // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1
@@ -126,7 +134,8 @@ struct Params {
   int M, N, K;
   int n_tiles, num_tiles, k_stages;
   int ksteps_total;  // K / 64
-  int stall_group;   // test hook: this CTA group's MMA warp stops after 3 stages (-1: none)
+  int stall_group;   // test hook: CTA group that stalls (-1: none) ...
+  int stall_mode;    // ... 1: its MMA warp stops after 3 stages; 2: its second CTA's producer stops after 2
 };
 
 // Epilogue mode 1: instead of y, emit the next layer's NVFP4 input
@@ -151,6 +160,39 @@ struct EpiSel {
 template <>
 struct EpiSel<1> {
   using type = EpiQuant;
+};
+
+// Prologue mode 1: the activations x [M, K] arrive in BF16 and the kernel
+// quantizes them itself.  Two warps of every CTA walk the quantization items
+// (32 rows x 64 columns each) in row-block order and write the codes and
+// tensor-core-layout scales to global memory (outputs the caller owns; they
+// stay in L2 for the tiles that read them), then count the item in the row
+// block's ready counter.  A producer loads a row block's A tiles only once
+// its counter has seen all 4 * K/64 items.  All CTAs of the grid are resident
+// at once (the grid is sized to the clusters that fit), so every item a
+// producer waits for is being worked on.  The counters start at zero; the
+// last CTA to leave sets them back to zero.
+struct ProQuant {
+  QuantTable tab;     // decision table of the activations' global scale
+  const uint16_t* x;  // BF16 [M, K], rows ldx elements apart
+  uint8_t* codes;     // [M, K/2]
+  uint8_t* scales;    // tensor-core layout of [M, K]
+  unsigned long long* clip;  // may be null
+  uint32_t* sync;     // n_rb ready counters, then the exit counter
+  int64_t ldx;
+  float inv6sg;
+  uint32_t clip_thr;
+  int katoms;  // K / 64
+  int n_rb;    // ceil(M / 128)
+};
+struct ProNone {};
+template <int kPro>
+struct ProSel {
+  using type = ProNone;
+};
+template <>
+struct ProSel<1> {
+  using type = ProQuant;
 };
 
 
@@ -230,6 +272,28 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity) {
     if ((i & 255u) == 0u && global_ns() - t0 > kDrainLimitNs) break;
   }
   atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+}
+
+// Wait for the peer producer's end-of-loading report (an arrival with release
+// semantics at cluster scope).  The peer reports once its own waits have
+// ended, which can take one full wait limit after this CTA stopped, so this
+// waits for the wait limit plus the drain limit before giving up.
+__device__ __forceinline__ bool wait_report(uint32_t bar) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0; i < (1u << 30); ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255u) == 0u && global_ns() - t0 > kWaitLimitNs + kDrainLimitNs) break;
+  }
+  atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+  return false;
 }
 
 // Tensor TMA load into this CTA's shared memory.  kCta == 2: `bar` may be the
@@ -455,13 +519,112 @@ struct Ring {
   }
 };
 
-template <int kCta, int kEpi, int kBN>
-__global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
+// ---- prologue quantizer (kPro = 1) ----------------------------------------------
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.global.acquire.gpu.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait (about 4 s) until the counter reaches `target`; the whole warp
+// polls the same word.  The async proxy (the tensor copies that follow) then
+// sees what the counted items wrote.
+__device__ __forceinline__ bool wait_counter(const uint32_t* ctr, uint32_t target, volatile int* abort) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 0; i < (1u << 30); ++i) {
+    if (ld_acquire_u32(ctr) >= target) {
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      return true;
+    }
+    if (*abort) return false;
+    if ((i & 15u) == 15u && global_ns() - t0 > kWaitLimitNs) break;
+    __nanosleep(64);
+  }
+  atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+  *abort = 1;
+  return false;
+}
+
+// One quantization item: rows rb*128 + r1*32 .. +31, columns kc*64 .. +63 of
+// x.  Lane l holds rows r1*32 + (l >> 2) + 8 i (i = 0..3), block l & 3.
+struct ProItem {
+  uint32_t w[4][8];
+};
+
+__device__ __forceinline__ void pro_item_coords(const ProQuant& pq, int item, int& rb, int& r1, int& kc) {
+  const int per_rb = 4 * pq.katoms;
+  rb = item / per_rb;
+  const int rest = item - rb * per_rb;
+  r1 = rest / pq.katoms;
+  kc = rest - r1 * pq.katoms;
+}
+
+__device__ __forceinline__ void pro_load(const ProQuant& pq, int M, int item, int lane, ProItem& it) {
+  int rb, r1, kc;
+  pro_item_coords(pq, item, rb, r1, kc);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int row = rb * 128 + r1 * 32 + (lane >> 2) + 8 * i;
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    if (row < M) {
+      const uint4* src = reinterpret_cast<const uint4*>(pq.x + (int64_t)row * pq.ldx + kc * 64 + (lane & 3) * 16);
+      a = __ldcs(src);
+      b = __ldcs(src + 1);
+    }
+    it.w[i][0] = a.x; it.w[i][1] = a.y; it.w[i][2] = a.z; it.w[i][3] = a.w;
+    it.w[i][4] = b.x; it.w[i][5] = b.y; it.w[i][6] = b.z; it.w[i][7] = b.w;
+  }
+}
+
+__device__ __forceinline__ void pro_quantize_store(const ProQuant& pq, const QuantTable& tab, int M, int K, int item,
+                                                   int lane, ProItem& it, unsigned long long& clips) {
+  int rb, r1, kc;
+  pro_item_coords(pq, item, rb, r1, kc);
+  const int j = lane & 3;
+  uint8_t* atom = pq.scales + ((size_t)rb * pq.katoms + kc) * 512;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r0 = (lane >> 2) + 8 * i;
+    const int row = rb * 128 + r1 * 32 + r0;
+    uint32_t amax;
+    uint2 cd;
+    uint32_t sc = nvfp4::quantize_block_codes(tab, pq.inv6sg, it.w[i], amax, cd);
+    if (row < M) {
+      *reinterpret_cast<uint2*>(pq.codes + (size_t)row * (size_t)(K >> 1) + kc * 32 + j * 8) = cd;
+      clips += nvfp4::block_clips(it.w[i], amax, pq.clip_thr);
+    } else {
+      sc = 0;  // padding rows of the scale layout hold zero scales
+    }
+    const uint32_t pair = sc | (__shfl_down_sync(0xFFFFFFFFu, sc, 1) << 8);
+    const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
+    if (j == 0) *reinterpret_cast<uint32_t*>(atom + r0 * 16 + r1 * 4) = word;
+  }
+}
+
+// Items are taken in chunks of kProChunk consecutive items of one row block
+// (4 * K/64 items per row block, so a chunk never straddles two): within a
+// chunk the next item's loads are in flight while the current one is
+// quantized, and the chunk is published with one fence and one count.
+constexpr int kProChunk = 4;
+
+// Publish a chunk: every lane's stores, then kProChunk counts in the row
+// block's counter (release), visible to the tensor copies of any CTA.
+__device__ __forceinline__ void pro_publish(const ProQuant& pq, int rb, int lane) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) atomicAdd(pq.sync + rb, (uint32_t)kProChunk);
+}
+
+template <int kCta, int kEpi, int kBN, int kPro>
+__global__ void __launch_bounds__(Cfg<kCta, kBN, kPro>::kThreads, 1)
     nvfp4_linear_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                         const __grid_constant__ CUtensorMap tmY, const Params p,
-                        const __grid_constant__ typename EpiSel<kEpi>::type eq) {
-  using C = Cfg<kCta, kBN>;
+                        const __grid_constant__ typename EpiSel<kEpi>::type eq,
+                        const __grid_constant__ typename ProSel<kPro>::type pq) {
+  using C = Cfg<kCta, kBN, kPro>;
   constexpr int S = C::kStages;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -474,12 +637,19 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
   auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };  // each CTA: accumulator ready
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + C::kAccBufs + a); };  // leader: accumulator drained
   const uint32_t drain_bar = bar0 + 8u * (2 * S + 2 * C::kAccBufs);
+  const uint32_t report_bar = drain_bar + 8u;  // leader: the peer producer reported its stage count
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffBar + C::kNumBars * 8);
+  volatile uint32_t* peer_issued = reinterpret_cast<volatile uint32_t*>(smem + C::kOffBar + C::kNumBars * 8 + 12);
   if constexpr (kEpi == 1) {
     // The next layer's decision table, in the (otherwise unused) output staging area.
     static_assert(sizeof(QuantTable) <= C::kEpiWarps * C::kEpiBufs * kEpiBufBytes, "table fits the staging area");
     const uint4* src = reinterpret_cast<const uint4*>(&eq.tab);
     uint4* dst = reinterpret_cast<uint4*>(smem + C::kOffEpi);
+    for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 16); i += blockDim.x) dst[i] = src[i];
+  }
+  if constexpr (kPro == 1) {
+    const uint4* src = reinterpret_cast<const uint4*>(&pq.tab);
+    uint4* dst = reinterpret_cast<uint4*>(smem + C::kOffQTab);
     for (int i = threadIdx.x; i < (int)(sizeof(QuantTable) / 16); i += blockDim.x) dst[i] = src[i];
   }
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffBar + C::kNumBars * 8 + 8);
@@ -501,6 +671,7 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
       mbar_init(acce_bar(a), C::kEpiWarps * kCta);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(report_bar, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
@@ -535,6 +706,7 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
     {
       Ring st;
       bool ok = true;
+      uint32_t issued = 0;  // stages this CTA has issued
       for (int t = pair; t < p.num_tiles && ok; t += npairs) {
         const int m_tile = t / p.n_tiles, n_tile = t % p.n_tiles;
         const int arow = m_tile * C::BM + (int)rank * 128;   // this CTA's A rows
@@ -542,7 +714,21 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
         const int brow = n0 + (int)rank * C::kBRows;          // this CTA's W rows
         const int ablk = arow / 128;  // this CTA's scale block of A
         const int jb0 = n0 / 128;      // first of the tile's two scale blocks of W
+        if constexpr (kPro == 1) {
+          // The row block's codes and scales are written by the grid's quantizer warps.
+          if (ablk < pq.n_rb && !wait_counter(pq.sync + ablk, 4u * (uint32_t)pq.katoms, abort_flag)) {
+            ok = false;
+            break;
+          }
+        }
         for (int kt = 0; kt < p.k_stages; ++kt) {
+          if (kCta == 2 && rank == 1 && pair == p.stall_group && p.stall_mode == 2 && issued == 2) {
+            // Test hook: this CTA stops loading, as if a wait had timed out, so
+            // the pair's loads of the same stage are left half issued.
+            atomicOr(&g_device_error, (unsigned)kDevErrTimeout);
+            ok = false;
+            break;
+          }
           if (!__all_sync(0xFFFFFFFFu, wait_bounded(empty_bar(st.slot), st.phase ^ 1u, abort_flag))) {
             ok = false;
             break;
@@ -561,13 +747,47 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
           }
           __syncwarp();
           st.next(S);
+          ++issued;
         }
       }
-      // Drain: the leader sees every load of both CTAs land on its stage
-      // barriers (the peer stays resident until the closing cluster barrier).
-      for (int s = 0; s < S; ++s) {
-        const uint32_t par = (s < st.slot) ? st.phase : (st.phase ^ 1u);
-        if (leader) wait_drain(full_bar(s), par);
+      // End of loading.  A pair's copies of a stage all complete on the leader's
+      // barrier of that stage, which counts one arrival per CTA, so the leader
+      // can see every copy of both CTAs land -- once it knows how many stages
+      // each CTA issued.  After a timeout the two may have stopped at
+      // different stages; the other CTA is told to stop too, the peer reports
+      // its count, and the leader arrives in the place of whichever CTA did
+      // not issue a stage, so that every issued stage's phase completes when
+      // its bytes have landed.  The peer stays resident until the closing
+      // cluster barrier, which the leader reaches only after this drain.
+      if (kCta == 2 && !ok && lane == 0)
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(map_to_rank(smem_u32((const void*)abort_flag), rank ^ 1u)),
+                     "r"(1u)
+                     : "memory");
+      uint32_t last = issued;
+      if (kCta == 2 && !leader) {
+        if (lane == 0) {
+          asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(map_to_rank(smem_u32((const void*)peer_issued), 0)),
+                       "r"(issued)
+                       : "memory");
+          asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(map_to_rank(report_bar, 0))
+                       : "memory");
+        }
+        __syncwarp();
+      } else if (kCta == 2) {
+        uint32_t reported = issued;
+        if (wait_report(report_bar)) reported = *peer_issued;
+        const uint32_t lo = min(issued, reported), hi = max(issued, reported);
+        if (lane == 0)
+          for (uint32_t i = lo; i < hi; ++i)
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(full_bar((int)(i % S))) : "memory");
+        __syncwarp();
+        last = hi;
+      }
+      if (leader) {
+        // The last use of every slot: stage i of slot i % S, phase (i / S) & 1.
+        const int slot = (int)(last % S);
+        const uint32_t phase = (last / S) & 1u;
+        for (int s = 0; s < S; ++s) wait_drain(full_bar(s), (s < slot) ? phase : (phase ^ 1u));
       }
     }
   } else if (warp == 1) {
@@ -589,13 +809,14 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
         // W scales start at column 0 or 2 of the 8 copied per K step (a
         // 256-row tile always at 0).
         const uint32_t sfb_shift = (uint32_t)(((t % p.n_tiles) * BN) % 128) / 32u;
+        constexpr uint32_t idesc = C::kIdesc;
         for (int kt = 0; kt < p.k_stages; ++kt) {
           const bool landed = wait_bounded(full_bar(st.slot), st.phase, abort_flag);
           if (!__all_sync(0xFFFFFFFFu, landed)) {
             ok = false;
             break;
           }
-          if (pair == p.stall_group && t == pair && kt == 3) {
+          if (pair == p.stall_group && p.stall_mode == 1 && t == pair && kt == 3) {
             // Test hook: stop issuing without committing, so every other role
             // of this group runs into its bounded wait and takes the drain path.
             ok = false;
@@ -623,11 +844,11 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
 #pragma unroll
               for (int k = 0; k < kKSteps; ++k)
                 tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
-                             C::kIdesc, (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
+                             idesc, (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
             } else {
               for (int k = 0; k < ks; ++k)
                 tc_mma<kCta>(d_tmem, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
-                             C::kIdesc, (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
+                             idesc, (kt | k) != 0 ? 1u : 0u, sf_tmem + 4 * k, sf_tmem + 4 * kKSteps + 8 * k + sfb_shift);
             }
             tc_commit<kCta>(empty_bar(st.slot));  // the stage's shared memory (both CTAs), once read
           }
@@ -653,13 +874,38 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
       __syncwarp();
       wait_drain(drain_bar, 0);
     }
+  } else if (kPro == 1 && warp < C::kEpiWarp0) {
+    // ===================== prologue quantizer (every CTA) =====================
+    if constexpr (kPro == 1) {
+      const QuantTable& tab = *reinterpret_cast<const QuantTable*>(smem + C::kOffQTab);
+      const int qw = (int)blockIdx.x * C::kQuantWarps + (warp - 2);
+      const int nqw = (int)gridDim.x * C::kQuantWarps;
+      const int n_chunks = pq.n_rb * 4 * pq.katoms / kProChunk;
+      unsigned long long clips = 0;
+      for (int ch = qw; ch < n_chunks; ch += nqw) {
+        if (*abort_flag) break;
+        const int item0 = ch * kProChunk;
+        ProItem cur, nxt;
+        pro_load(pq, p.M, item0, lane, cur);
+#pragma unroll 1
+        for (int k = 0; k < kProChunk; ++k) {
+          if (k + 1 < kProChunk) pro_load(pq, p.M, item0 + k + 1, lane, nxt);  // the next item's loads in flight
+          pro_quantize_store(pq, tab, p.M, p.K, item0 + k, lane, cur, clips);
+          cur = nxt;
+        }
+        pro_publish(pq, item0 / (4 * pq.katoms), lane);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) clips += __shfl_xor_sync(0xFFFFFFFFu, clips, o);
+      if (lane == 0 && clips != 0 && pq.clip != nullptr) atomicAdd(pq.clip, clips);
+    }
   } else {
     // ===================== epilogue (every CTA) =====================
-    // Warp ew = warp - 2 reads TMEM lane quadrant warp % 4 (32 output rows)
-    // and accumulator columns [hcol, hcol + kWarpCols).
+    // Warp ew = warp - kEpiWarp0 reads TMEM lane quadrant warp % 4 (32 output
+    // rows) and accumulator columns [hcol, hcol + kWarpCols).
     constexpr int kWarpCols = C::kWarpCols;
     constexpr int kChunks = kWarpCols / kEpiCols;
-    const int ew = warp - 2;
+    const int ew = warp - C::kEpiWarp0;
     const int q = warp & 3;
     const int hcol = (ew >> 2) * kWarpCols;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -794,16 +1040,6 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (kCta == 2 && *abort_flag != 0 && threadIdx.x == 0) {
-    // After a timeout the two producers may have stopped at different stages,
-    // and a peer's A/W copies complete on the leader's barriers, which this CTA
-    // cannot observe.  Give any such copy time to land before either CTA
-    // retires (copies take microseconds; this waits 2 ms).
-    const uint64_t t0 = global_ns();
-    while (global_ns() - t0 < 2000000ull) {
-    }
-  }
-  __syncthreads();
   if (kCta == 2) cluster_sync();  // the peer no longer needs this CTA's shared memory or TMEM
   tc_fence_after();
   if (warp == 1) {
@@ -812,6 +1048,20 @@ __global__ void __launch_bounds__(Cfg<kCta, kBN>::kThreads, 1)
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
     else
       asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+  }
+  if constexpr (kPro == 1) {
+    // Every producer of this CTA is done with the counters.  The last CTA to
+    // get here sets them back to zero for the next launch.
+    __shared__ int last_cta;
+    if (threadIdx.x == 0) {
+      __threadfence();
+      last_cta = atomicAdd(pq.sync + pq.n_rb, 1u) == gridDim.x - 1;
+    }
+    __syncthreads();
+    if (last_cta) {
+      __threadfence();
+      for (int i = threadIdx.x; i <= pq.n_rb; i += blockDim.x) pq.sync[i] = 0u;
+    }
   }
 }
 
@@ -825,6 +1075,89 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
   mbar_init(smem_u32(&bar), 1);
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   wait_bounded(smem_u32(&bar), 0, &abort_flag, limit_ns);
+}
+
+// Tensor-pipe rate probe (a measurement, not part of the layer): every CTA pair
+// of the grid issues `iters` rounds of four tcgen05.mma cta_group::2
+// kind::mxf4nvf4 block_scale (256 x 256 x 64 each, the GEMM's instruction and
+// tile) on operands resident in shared memory -- no global memory traffic --
+// optionally preceded, as in the GEMM's mainloop, by the twelve tcgen05.cp
+// scale copies of a stage into alternating TMEM scale buffers.  Timed by the
+// host around the launch, it gives the FP4 tensor rate the GEMM can reach.
+constexpr int kProbeThreads = 128;
+constexpr int kProbeSmem = 160 * 1024;  // one CTA per SM, so the pairs never wait on each other for TMEM
+__global__ void __launch_bounds__(kProbeThreads, 1) mma_rate_probe_kernel(int iters, int with_copies) {
+  using C = Cfg<2, 256>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ uint64_t done_bar;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int abort_flag;
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t rank = cluster_rank();
+  // Operands: A 16 KB, W 16 KB (128-byte swizzled tiles), scale atoms 2 + 4 KB.
+  // Pseudo-random codes; scales drawn from E4M3 codes 0x28 .. 0x47 (about 0.25 .. 4).
+  for (int i = threadIdx.x; i < (38 * 1024) / 4; i += blockDim.x) {
+    uint32_t h = (uint32_t)i * 0x9E3779B1u + (blockIdx.x + 1) * 0x85EBCA6Bu;
+    h ^= h >> 15;
+    h *= 0x2C1B3C6Du;
+    h ^= h >> 12;
+    if (i >= 8192) h = 0x28282828u + (h & 0x1F1F1F1Fu);
+    reinterpret_cast<uint32_t*>(smem)[i] = h;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&done_bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_proxy_async_smem();
+  if ((threadIdx.x >> 5) == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&tmem_slot)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_slot;
+  if ((threadIdx.x >> 5) == 0 && rank == 0) {
+    const uint64_t adesc = smem_desc(sbase, true), bdesc = smem_desc(sbase + kABytes, true);
+    const uint32_t sfa_s = sbase + 2 * kABytes, sfb_s = sfa_s + kSFABytes;
+    for (int it = 0; it < iters; ++it) {
+      const uint32_t sf_tmem = tmem_base + (uint32_t)(C::kSfCol0 + (it & 1) * kSfCols);
+      if (elect_one()) {
+        if (with_copies || it == 0) {  // without copies, the scales are copied once, before the first round
+#pragma unroll
+          for (int k = 0; k < kKSteps; ++k) {
+            tc_cp_atom<2>(sf_tmem + 4 * k, smem_desc(sfa_s + k * kAtomBytes, false));
+            tc_cp_atom<2>(sf_tmem + 4 * kKSteps + 8 * k, smem_desc(sfb_s + k * kAtomBytes, false));
+            tc_cp_atom<2>(sf_tmem + 4 * kKSteps + 8 * k + 4, smem_desc(sfb_s + (kKSteps + k) * kAtomBytes, false));
+          }
+        }
+        const uint32_t sf = (with_copies || it == 0) ? sf_tmem : tmem_base + (uint32_t)C::kSfCol0;
+#pragma unroll
+        for (int k = 0; k < kKSteps; ++k)
+          tc_mma<2>(tmem_base, adesc + (uint64_t)(k * (kMmaK / 2) / 16), bdesc + (uint64_t)(k * (kMmaK / 2) / 16),
+                    C::kIdesc, (it | k) != 0 ? 1u : 0u, sf + 4 * k, sf + 4 * kKSteps + 8 * k);
+      }
+      __syncwarp();
+    }
+    if (elect_one()) tc_commit<2>(smem_u32(&done_bar));  // arrives in both CTAs
+    __syncwarp();
+  }
+  if (threadIdx.x == 0) {
+    // Every MMA this pair issued has completed before TMEM is released.
+    if (!wait_bounded(smem_u32(&done_bar), 0, &abort_flag)) wait_drain(smem_u32(&done_bar), 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  if ((threadIdx.x >> 5) == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols));
+  }
 }
 
 // ---- host side ----------------------------------------------------------------
@@ -847,12 +1180,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Test hook: FH_GEMM_TEST_STALL=1 makes CTA group 0's MMA warp stop after three
-// stages of its first tile (when K spans at least four stages), so that the
-// kernel's bounded waits expire and the call ends with FH_ERR_TIMEOUT.
-int stall_group() {
+// Test hooks (CTA group 0 only): FH_GEMM_TEST_STALL=1 makes the MMA warp stop
+// after three stages of its first tile (when K spans at least four stages), so
+// that the kernel's bounded waits expire; FH_GEMM_TEST_STALL=2 makes the second
+// CTA of the pair stop loading after two stages, so that the two producers end
+// at different stages.  Either way the call ends with FH_ERR_TIMEOUT.
+int stall_mode() {
   const char* e = getenv("FH_GEMM_TEST_STALL");  // read per launch, so a test can switch it off again
-  return (e != nullptr && e[0] == '1') ? 0 : -1;
+  return (e != nullptr && (e[0] == '1' || e[0] == '2') && e[1] == 0) ? e[0] - '0' : 0;
 }
 
 // Which kernel form to run: the CTA pair (default) or single CTAs.  The
@@ -878,17 +1213,18 @@ int tile_width(int64_t N) {
   return 256;
 }
 
-template <int kCta, int kEpi, int kBN>
+template <int kCta, int kEpi, int kBN, int kPro = 0>
 cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmSA,
                         const CUtensorMap& tmSB, const CUtensorMap& tmY, const Params& p,
-                        const typename EpiSel<kEpi>::type& eq, cudaStream_t s) {
-  using C = Cfg<kCta, kBN>;
+                        const typename EpiSel<kEpi>::type& eq, cudaStream_t s,
+                        const typename ProSel<kPro>::type& pq = typename ProSel<kPro>::type()) {
+  using C = Cfg<kCta, kBN, kPro>;
   static DeviceTable groups_of;  // resident CTA groups of this form, per device
   int dev = 0;
   cudaGetDevice(&dev);
   const int max_groups = per_device(groups_of, dev, [](int) {
-    cudaError_t e =
-        cudaFuncSetAttribute(nvfp4_linear_kernel<kCta, kEpi, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
+    cudaError_t e = cudaFuncSetAttribute(nvfp4_linear_kernel<kCta, kEpi, kBN, kPro>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemAlloc);
     if (e != cudaSuccess) return -(int)e;
     int max_groups = sm_count() / kCta;
     if (kCta == 2) {
@@ -905,7 +1241,7 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4_linear_kernel<2, kEpi, kBN>, &cfg) == cudaSuccess &&
+      if (cudaOccupancyMaxActiveClusters(&clusters, nvfp4_linear_kernel<2, kEpi, kBN, kPro>, &cfg) == cudaSuccess &&
           clusters > 0)
         max_groups = clusters < max_groups ? clusters : max_groups;
       cudaGetLastError();
@@ -913,7 +1249,9 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
     return max_groups > 0 ? max_groups : 1;
   });
   if (max_groups <= 0) return (cudaError_t)(-max_groups);
-  const int groups = p.num_tiles < max_groups ? p.num_tiles : max_groups;
+  // The quantizing prologue spreads its items over every resident pair, so it
+  // launches them all even when there are fewer tiles.
+  const int groups = (kPro == 1 || p.num_tiles >= max_groups) ? max_groups : p.num_tiles;
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[2];
   int nattr = 0;
@@ -931,7 +1269,7 @@ cudaError_t launch_form(const CUtensorMap& tmA, const CUtensorMap& tmB, const CU
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = nattr;
-  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi, kBN>, tmA, tmB, tmSA, tmSB, tmY, p, eq);
+  return cudaLaunchKernelEx(&cfg, nvfp4_linear_kernel<kCta, kEpi, kBN, kPro>, tmA, tmB, tmSA, tmSB, tmY, p, eq, pq);
 }
 
 }  // namespace
@@ -947,6 +1285,48 @@ bool make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* ba
   const cuuint32_t estr[2] = {1, 1};
   return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_mma_rate_probe(int iters, int with_copies, int* pairs_out, cudaStream_t s) {
+  static DeviceTable pairs_of;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int pairs = per_device(pairs_of, dev, [](int) {
+    cudaError_t e = cudaFuncSetAttribute(mma_rate_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kProbeSmem);
+    if (e != cudaSuccess) return -(int)e;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2 * (sm_count() / 2));
+    cfg.blockDim = dim3(kProbeThreads);
+    cfg.dynamicSmemBytes = kProbeSmem;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, mma_rate_probe_kernel, &cfg) != cudaSuccess || clusters < 1)
+      clusters = sm_count() / 2;
+    cudaGetLastError();
+    return clusters < sm_count() / 2 ? clusters : sm_count() / 2;
+  });
+  if (pairs <= 0) return (cudaError_t)(-pairs);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kProbeThreads);
+  cfg.dynamicSmemBytes = kProbeSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  *pairs_out = pairs;
+  return cudaLaunchKernelEx(&cfg, mma_rate_probe_kernel, iters, with_copies);
 }
 
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t s) {
@@ -971,9 +1351,10 @@ namespace {
 // y is the BF16 output (mode 0) or null (mode 1, outputs in *eq).
 cudaError_t launch_linear(const uint8_t* a_codes, const uint8_t* a_scales, float a_g, const uint8_t* w_codes,
                           const uint8_t* w_scales, float w_g, const uint16_t* bias, uint16_t* y, int64_t M,
-                          int64_t N, int64_t K, const EpiQuant* eq, cudaStream_t s, const char** why) {
-  const int ctas = cta_mode();
-  const int BN = ctas == 2 ? tile_width(N) : 192;
+                          int64_t N, int64_t K, const EpiQuant* eq, cudaStream_t s, const char** why,
+                          const ProQuant* pq = nullptr) {
+  const int ctas = pq != nullptr ? 2 : cta_mode();
+  const int BN = pq != nullptr ? 256 : (ctas == 2 ? tile_width(N) : 192);
   CUtensorMap tmA, tmB, tmY;
   const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
   if (!make_tensor_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_codes, (uint64_t)K / 2, (uint64_t)M,
@@ -1010,7 +1391,13 @@ cudaError_t launch_linear(const uint8_t* a_codes, const uint8_t* a_scales, float
   p.num_tiles = m_tiles * p.n_tiles;
   p.k_stages = (int)((K + BK - 1) / BK);
   p.ksteps_total = (int)(K / kMmaK);
-  p.stall_group = stall_group();
+  p.stall_mode = stall_mode();
+  p.stall_group = p.stall_mode != 0 ? 0 : -1;
+  if (pq != nullptr) {
+    p.stall_group = -1;
+    p.stall_mode = 0;
+    return launch_form<2, 0, 256, 1>(tmA, tmB, tmSA, tmSB, tmY, p, EpiNone(), s, *pq);
+  }
   if (eq == nullptr) {
     const EpiNone none;
     if (ctas == 1) return launch_form<1, 0, 192>(tmA, tmB, tmSA, tmSB, tmY, p, none, s);
@@ -1029,6 +1416,26 @@ cudaError_t launch_nvfp4_linear(const uint8_t* a_codes, const uint8_t* a_scales,
                                 const uint16_t* bias, uint16_t* y, int64_t M, int64_t N, int64_t K,
                                 cudaStream_t s, const char** why) {
   return launch_linear(a_codes, a_scales, a_g, w_codes, w_scales, w_g, bias, y, M, N, K, nullptr, s, why);
+}
+
+cudaError_t launch_nvfp4_linear_quant_prologue(const uint16_t* x, int64_t ldx, float a_g, const uint8_t* w_codes,
+                                               const uint8_t* w_scales, float w_g, const uint16_t* bias, uint16_t* y,
+                                               uint8_t* a_codes, uint8_t* a_scales, unsigned long long* clip,
+                                               uint32_t* sync, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                                               const char** why) {
+  static thread_local ProQuant pq;  // 3 KB: kept off the stack
+  memcpy(&pq.tab, &quant_table_for(a_g), sizeof(QuantTable));
+  pq.x = x;
+  pq.codes = a_codes;
+  pq.scales = a_scales;
+  pq.clip = clip;
+  pq.sync = sync;
+  pq.ldx = ldx;
+  pq.inv6sg = (float)(1.0 / (6.0 * (double)a_g));
+  pq.clip_thr = clip_threshold_bits(a_g);
+  pq.katoms = (int)(K / 64);
+  pq.n_rb = (int)((M + 127) / 128);
+  return launch_linear(a_codes, a_scales, a_g, w_codes, w_scales, w_g, bias, y, M, N, K, nullptr, s, why, &pq);
 }
 
 cudaError_t launch_nvfp4_linear_gelu_quant(const uint8_t* a_codes, const uint8_t* a_scales, float a_g,

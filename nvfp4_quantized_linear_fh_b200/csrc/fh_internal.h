@@ -77,6 +77,12 @@ cudaError_t launch_scales_to_rowmajor(const uint8_t* tiled, uint8_t* rowmajor, i
                                       int64_t K, cudaStream_t s);
 cudaError_t launch_gelu(const uint16_t* x, uint16_t* y, int64_t n, cudaStream_t s);
 
+// Tensor-pipe rate probe (fh_gemm.cu): every resident CTA pair issues `iters`
+// rounds of four 256 x 256 x 64 block-scaled FP4 MMAs from shared memory
+// (with_copies: each round preceded by the GEMM's twelve scale copies);
+// *pairs_out receives the number of pairs launched.
+cudaError_t launch_mma_rate_probe(int iters, int with_copies, int* pairs_out, cudaStream_t s);
+
 // One-thread kernel whose bounded wait runs out after limit_ns (fh_gemm.cu).
 cudaError_t launch_bounded_wait_selftest(uint64_t limit_ns, cudaStream_t s);
 
@@ -96,6 +102,18 @@ cudaError_t launch_nvfp4_linear_gelu_quant(const uint8_t* a_codes, const uint8_t
                                            const uint16_t* bias, float out_g, uint8_t* out_codes,
                                            uint8_t* out_scales, unsigned long long* out_clip, int64_t M,
                                            int64_t N, int64_t K, cudaStream_t s, const char** why);
+
+// The GEMM with the activations' quantization fused into the kernel: x BF16
+// [M, K] (rows ldx elements apart) is quantized with global scale a_g by two
+// warps of every CTA into a_codes [M, K/2] and tensor-core-layout a_scales
+// (outputs), which the same kernel's tiles read once each row block is done;
+// sync: ceil(M / 128) + 1 words, zero at launch and zero again at exit.
+// Clipped elements of x are added to *clip (if not null).
+cudaError_t launch_nvfp4_linear_quant_prologue(const uint16_t* x, int64_t ldx, float a_g, const uint8_t* w_codes,
+                                               const uint8_t* w_scales, float w_g, const uint16_t* bias, uint16_t* y,
+                                               uint8_t* a_codes, uint8_t* a_scales, unsigned long long* clip,
+                                               uint32_t* sync, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                                               const char** why);
 
 // INT8 query/key path (fh_int8.cu).  Arguments are validated by the caller.
 // Per-row symmetric INT8 quantization of BF16 rows (d % 8 == 0).

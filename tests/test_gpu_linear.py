@@ -257,20 +257,24 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     m.fh_device_status()
 
 
-def test_gemm_stall_times_out_drains_and_context_survives(monkeypatch):
-    """With the test hook FH_GEMM_TEST_STALL=1 the first CTA pair's MMA warp
-    stops issuing after three stages of its first tile, without committing.
-    That pair's producer and epilogue then run into their
-    bounded waits (about 4 s) while copies and MMAs are in flight; the kernel
-    drains them and frees TMEM, and the host reads FH_ERR_TIMEOUT.  With the
-    hook off, the next GEMM in the same context passes parity."""
+@pytest.mark.parametrize("mode", ["1", "2"])
+def test_gemm_stall_times_out_drains_and_context_survives(monkeypatch, mode):
+    """Test hook FH_GEMM_TEST_STALL=1: the first CTA pair's MMA warp stops
+    issuing after three stages of its first tile, without committing; that
+    pair's producers and epilogues run into their bounded waits (about 4 s)
+    with copies and MMAs in flight.  FH_GEMM_TEST_STALL=2: the pair's second
+    CTA stops loading after two stages, so its producer and the leader's end at
+    different stages and the leader must account for the stages only it
+    issued.  Either way the kernel drains what it issued and frees TMEM, and
+    the host reads FH_ERR_TIMEOUT; with the hook off, the next GEMM in the same
+    context passes parity."""
     m = fh()
     m.fh_device_status()                      # clean start
     x = S.random_bf16(("stall", "x"), (1024, 2688), 1.0)
     w = S.random_bf16(("stall", "w"), (1344, 2688), 0.02)
     sg_a = oracle.scale_from_amax(oracle.amax(x))
     sg_w = oracle.scale_from_amax(oracle.amax(w))
-    monkeypatch.setenv("FH_GEMM_TEST_STALL", "1")
+    monkeypatch.setenv("FH_GEMM_TEST_STALL", mode)
     run_layer(x, w, None, sg_a, sg_w)
     monkeypatch.delenv("FH_GEMM_TEST_STALL")
     with pytest.raises(m.FHError) as e:
