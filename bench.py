@@ -158,26 +158,10 @@ def bench_fh(args, rank, world, local_rank):
     S, layer = make_inputs(rank, args.M, args.quick)
     M, K, N = layer.M, layer.K, layer.N
 
-    def to_dev(bits):
-        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
-
-    # --- offline: calibration, weight quantization (not timed) ---
-    x_bits = S.activations(layer)
-    x = to_dev(x_bits)
-    amax = torch.zeros(1, dtype=torch.float32, device=dev)
-    fh.fh_amax(x, amax)
-    chunk = 64
-    for b0 in range(layer.n_eval_batches, layer.n_calib, chunk):
-        nb = min(chunk, layer.n_calib - b0)
-        fh.fh_amax(to_dev(S.activation_batches(layer, b0, nb)), amax)
-    sg_a = fh.fh_scale_from_amax(amax.item())
-    w = to_dev(S.weights(layer))
-    wamax = torch.zeros(1, dtype=torch.float32, device=dev)
-    fh.fh_amax(w, wamax)
-    sg_w = fh.fh_scale_from_amax(wamax.item())
-    wc, wsc = fh.empty_quantized(N, K, device=dev)
-    fh.fh_quantize_act(w, sg_w, wc, wsc, None)
-    bias = to_dev(S.bias(layer))
+    # --- offline: inputs drawn on the GPU, calibration, weight quantization (not timed) ---
+    x, sg_a = _dev_inputs(fh, S, layer, M, dev, calib=layer.n_calib)
+    wc, wsc, sg_w, bias, w = _dev_weights(fh, S, layer, dev)
+    x_bits, w_bits, b_bits = _bits(x[:CPU_SAMPLE_ROWS]), _bits(w), _bits(bias)
     del w
 
     ac, asc = fh.empty_quantized(M, K, device=dev)
@@ -218,6 +202,27 @@ def bench_fh(args, rank, world, local_rank):
     fh.fh_device_status()
     clips = int(clip.item())
 
+    # --- the quantization fused into the GEMM (one launch), timed the same way ---
+    t_fused = []
+    if not args.no_fused:
+        sync = fh.empty_fused_sync(M, device=dev)
+        yf = torch.empty_like(y)
+        acf, ascf = fh.empty_quantized(M, K, device=dev)
+        for _ in range(args.warmup):
+            fh.fh_nvfp4_linear_fused_quant(x, sg_a, wc, wsc, sg_w, bias, yf, acf, ascf, None, sync)
+        torch.cuda.synchronize()
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(args.steps, 50))]
+        for e in fev:
+            e[0].record(stream)
+            fh.fh_nvfp4_linear_fused_quant(x, sg_a, wc, wsc, sg_w, bias, yf, acf, ascf, None, sync)
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        fh.fh_device_status()
+        t_fused = [e[0].elapsed_time(e[1]) * 1e-3 for e in fev]
+        if not torch.equal(yf.view(torch.int16), y.view(torch.int16)):
+            raise RuntimeError("the fused path's output differs from the two separate calls")
+        del sync, yf, acf, ascf
+
     # --- end to end through the public API with host buffers ---
     # fh_nvfp4_linear_host: pinned BF16 x in host memory -> BF16 y in host
     # memory, the upload, kernels and download pipelined over 4096-row chunks.
@@ -247,13 +252,33 @@ def bench_fh(args, rank, world, local_rank):
         from nvfp4_quantized_linear_fh_b200 import dist as fhd
         t_step, t_e2e = fhd.max_over_ranks([t_step, t_e2e], device=dev)
     flops = 2.0 * M * N * K
-    return dict(t_step=t_step, t_quant=t_quant, t_gemm=t_gemm, t_e2e=t_e2e, e_steps=e_steps, flops=flops,
+    return dict(t_step=t_step, t_quant=t_quant, t_gemm=t_gemm, t_e2e=t_e2e, e_steps=e_steps, flops=flops, t_fused=t_fused,
                 clips=clips, sampler=sampler.summary(), M=M, N=N, K=K,
-                h2d=M * K * 2, d2h=M * N * 2, x_bits=x_bits, w_bits=S.weights(layer), b_bits=S.bias(layer),
+                h2d=M * K * 2, d2h=M * N * 2, x_bits=x_bits, w_bits=w_bits, b_bits=b_bits,
                 sg_a=sg_a, sg_w=sg_w)
 
 
 _WQ_CACHE = {}
+
+
+def fp4_tensor_rate(with_copies: bool, iters: int = 60000, reps: int = 3) -> float:
+    """FLOP/s of the library's tensor-rate probe: every CTA pair issues `iters`
+    rounds of four 256 x 256 x 64 block-scaled FP4 MMAs from shared memory
+    (with_copies: plus the GEMM's twelve scale copies per round), timed with
+    CUDA events; the best of `reps` launches after a warm-up."""
+    import torch
+    import nvfp4_quantized_linear_fh_b200 as fh
+    fh.fh_selftest_mma_rate(2000, with_copies)
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        pairs = fh.fh_selftest_mma_rate(iters, with_copies)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, pairs * iters * 2.0 * 256 ** 3 / (e0.elapsed_time(e1) * 1e-3))
+    fh.fh_device_status()
+    return best
 
 
 def gemm_bytes(M, N, K):
@@ -381,6 +406,294 @@ def bench_ffn(args):
         "variants": {n: {"value": flops / t / 1e12, "ms_per_step": t * 1e3, "calls": variants[n][1]}
                      for n, t in times.items()},
         "outputs_bit_identical": identical}))
+
+
+# ---------------------------------------------------------------------------
+# The five synthetic configurations, each with its own roofline fractions and
+# its oracle baseline (the "configs" object of the default line, or one line
+# each with --workload tiny|attn_proj|ffn_pair|block_sweep).
+# ---------------------------------------------------------------------------
+
+def _dev_inputs(fh, S, layer, M, dev, calib):
+    """The layer's first M rows (BF16, drawn on the GPU) and its calibrated global scale:
+    amax over `calib` batches of its calibration stream (the input being their prefix)."""
+    import torch
+    nb = M // layer.batch
+    x = S.activation_batches_t(layer, 0, nb, dev).view(torch.bfloat16)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    fh.fh_amax(x, amax)
+    for b0 in range(nb, calib, 128):
+        n = min(128, calib - b0)
+        fh.fh_amax(S.activation_batches_t(layer, b0, n, dev).view(torch.bfloat16), amax)
+    return x, fh.fh_scale_from_amax(amax.item())
+
+
+def _dev_weights(fh, S, layer, dev):
+    """W drawn on the GPU and quantized offline with its own amax scale; the BF16 W is returned too."""
+    import torch
+    w = S.weights_t(layer, dev).view(torch.bfloat16)
+    wamax = torch.zeros(1, dtype=torch.float32, device=dev)
+    fh.fh_amax(w, wamax)
+    sg = fh.fh_scale_from_amax(wamax.item())
+    wc, wsc = fh.empty_quantized(layer.N, layer.K, device=dev)
+    fh.fh_quantize_act(w, sg, wc, wsc, None)
+    return wc, wsc, sg, S.bias_t(layer, dev).view(torch.bfloat16), w
+
+
+def _bits(t):
+    return t.view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+
+
+def _time_calls(calls, steps, warmup, flush=None):
+    """calls: [(tag, fn)] making one step.  Runs `warmup` untimed steps, then
+    `steps` steps with a CUDA event between consecutive calls (and `flush`, if
+    given, before each step, outside the events).  Returns ({tag: seconds per
+    step, summed over the tag's calls}, seconds of the whole timed region)."""
+    import torch
+    for _ in range(warmup):
+        if flush is not None:
+            flush()
+        for _, fn in calls:
+            fn()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        ev[0].record()
+        for i, (_, fn) in enumerate(calls):
+            fn()
+            ev[i + 1].record()
+        evs.append(ev)
+    torch.cuda.synchronize()
+    out = {}
+    for ev in evs:
+        for i, (tag, _) in enumerate(calls):
+            out[tag] = out.get(tag, 0.0) + ev[i].elapsed_time(ev[i + 1]) * 1e-3
+    region = sum(out.values())
+    return {k: v / steps for k, v in out.items()}, region
+
+
+def _gemm_roof(flops, secs, pk, sustained):
+    burst, sust = pk["bf16"] * FP4_OVER_BF16, pk["bf16_sustained"] * FP4_OVER_BF16
+    ach = flops / secs / 1e12
+    peak = sust if sustained else burst
+    return {"bound": "tensor", "achieved": ach, "unit": "TFLOP/s", "peak": peak, "frac": ach / peak,
+            "peak_kind": "sustained" if sustained else "burst", "frac_of_burst_peak": ach / burst,
+            "frac_of_sustained_peak": ach / sust}
+
+
+def _quant_roof(M, K, secs, pk):
+    ach = QUANT_BYTES_PER_ELEM * M * K / secs / 1e9
+    return {"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": pk["hbm_gbs"], "frac": ach / pk["hbm_gbs"],
+            "us": secs * 1e6}
+
+
+def _oracle_layer_rate(x_bits, sg_a, wq, b_bits, rows):
+    """The oracle on `rows` token rows: quantize them, binary64 dequantized GEMM
+    against the already-quantized weights wq = (codes, scales, s_gW).
+    Returns (FLOP/s, seconds)."""
+    import oracle
+    wc, wsc, sg_w = wq
+    K, N = x_bits.shape[1], wc.shape[0]
+    t0 = time.perf_counter()
+    ac, asc, _ = oracle.quantize(x_bits[:rows], sg_a)
+    oracle.linear(ac, asc, sg_a, wc, wsc, sg_w, b_bits)
+    dt = time.perf_counter() - t0
+    return 2.0 * rows * N * K / dt, dt
+
+
+def _oracle_weights(w):
+    import oracle
+    wb = _bits(w)
+    sg = oracle.scale_from_amax(oracle.amax(wb))
+    c, s, _ = oracle.quantize(wb, sg)
+    return c, s, sg
+
+
+def measure_layer_config(name, fh, S, dev, pk, args):
+    """tiny (128 x 256 -> 256) or attn_proj (8192 x 2688 -> 2688): quantize + GEMM per
+    step; both fit in L2, so L2 is flushed (a 256 MB write) before every step."""
+    import torch
+    layer = S.workloads()[name][0]
+    M, K, N = layer.M, layer.K, layer.N
+    # Both recipes put one outlier of exactly 137 L in every batch, so the amax
+    # over the evaluation batches is the amax over the whole calibration stream.
+    x, sg_a = _dev_inputs(fh, S, layer, M, dev, calib=layer.n_eval_batches)
+    wc, wsc, sg_w, b, w = _dev_weights(fh, S, layer, dev)
+    ac, asc = fh.empty_quantized(M, K, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    clip = torch.zeros(1, dtype=torch.int64, device=dev)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)
+    calls = [("quant", lambda: fh.fh_quantize_act(x, sg_a, ac, asc, clip)),
+             ("gemm", lambda: fh.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, b, y))]
+    steps = 100
+    t, region = _time_calls(calls, steps, max(args.warmup, 3), flush=lambda: flush.fill_(1.0))
+    fh.fh_device_status()
+    flops = 2.0 * M * N * K
+    out = {"workload": f"{name} {M}x{K}->{N}", "M": M, "K": K, "N": N, "steps": steps,
+           "step_us": (t["quant"] + t["gemm"]) * 1e6, "tflops": flops / (t["quant"] + t["gemm"]) / 1e12,
+           "gemm_us": t["gemm"] * 1e6, "gemm_roofline": _gemm_roof(flops, t["gemm"], pk, False),
+           "quantizer_roofline": _quant_roof(M, K, t["quant"], pk), "clip_count": int(clip.item()),
+           "l2": "flushed before every step (256 MB write, outside the timed events)"}
+    if not args.no_cpu_baseline:
+        rows = M if M <= 128 else 32
+        rate, dt = _oracle_layer_rate(_bits(x), sg_a, _oracle_weights(w), _bits(b), rows)
+        out["cpu_baseline"] = {"value": rate / 1e12, "unit": "TFLOPS", "cores": len(os.sched_getaffinity(0)),
+                               "kind": "oracle", "sample": f"{rows} of the {M} token rows ({dt:.2f} s)"}
+    return out
+
+
+def measure_ffn_config(fh, S, dev, pk, args):
+    """Config 4, the FFN pair at 32768 tokens: up 2688 -> 10752, GELU, down 10752 -> 2688,
+    each layer's input quantized with its own calibrated scale (the down layer's
+    calibrated on the GELU outputs of the same batches).  Two paths on the same
+    operands: the plain chain (quantize, GEMM, GELU, quantize, GEMM) and the fused
+    one (quantize, GEMM with the GELU-quantizing epilogue, GEMM)."""
+    import torch
+    up, down = S.workloads()["ffn"]
+    M, K, N1, N2 = up.M, up.K, up.N, down.N
+    # The up layer's recipe has one outlier of exactly 137 L per batch: the amax
+    # over the evaluation batches is that of the whole stream.
+    x, sg_x = _dev_inputs(fh, S, up, M, dev, calib=up.n_eval_batches)
+    w1c, w1s, sg_w1, b1, w1 = _dev_weights(fh, S, up, dev)
+    w2c, w2s, sg_w2, b2, w2 = _dev_weights(fh, S, down, dev)
+    xc, xs = fh.empty_quantized(M, K, device=dev)
+    h = torch.empty((M, N1), dtype=torch.bfloat16, device=dev)
+    g = torch.empty_like(h)
+    gc, gs = fh.empty_quantized(M, N1, device=dev)
+    y = torch.empty((M, N2), dtype=torch.bfloat16, device=dev)
+    clip = torch.zeros(1, dtype=torch.int64, device=dev)
+    fh.fh_quantize_act(x, sg_x, xc, xs, clip)
+    fh.fh_nvfp4_linear(xc, xs, sg_x, w1c, w1s, sg_w1, b1, h)
+    fh.fh_gelu_bf16(h, g)
+    amax = torch.zeros(1, dtype=torch.float32, device=dev)
+    fh.fh_amax(g, amax)
+    sg_g = fh.fh_scale_from_amax(amax.item())
+    plain = [("quant_up", lambda: fh.fh_quantize_act(x, sg_x, xc, xs, clip)),
+             ("gemm_up", lambda: fh.fh_nvfp4_linear(xc, xs, sg_x, w1c, w1s, sg_w1, b1, h)),
+             ("gelu", lambda: fh.fh_gelu_bf16(h, g)),
+             ("quant_down", lambda: fh.fh_quantize_act(g, sg_g, gc, gs, clip)),
+             ("gemm_down", lambda: fh.fh_nvfp4_linear(gc, gs, sg_g, w2c, w2s, sg_w2, b2, y))]
+    fused = [("quant_up", lambda: fh.fh_quantize_act(x, sg_x, xc, xs, clip)),
+             ("gemm_up_gelu_quant", lambda: fh.fh_nvfp4_linear_gelu_quant(xc, xs, sg_x, w1c, w1s, sg_w1, b1, sg_g,
+                                                                         gc, gs, clip)),
+             ("gemm_down", lambda: fh.fh_nvfp4_linear(gc, gs, sg_g, w2c, w2s, sg_w2, b2, y))]
+    steps = 20
+    tp, _ = _time_calls(plain, steps, max(args.warmup, 3))
+    y_plain = y.clone()
+    clip.zero_()
+    tf, _ = _time_calls(fused, steps, max(args.warmup, 3))
+    fh.fh_device_status()
+    identical = bool(torch.equal(y.view(torch.int16), y_plain.view(torch.int16)))
+    f_up, f_down = 2.0 * M * K * N1, 2.0 * M * N1 * N2
+    t_plain, t_fused = sum(tp.values()), sum(tf.values())
+    out = {"workload": f"FFN pair {M}x{K}->{N1} (GELU) ->{N2}", "M": M, "K": K, "N_up": N1, "N_down": N2,
+           "steps": steps, "block_ms_plain": t_plain * 1e3, "block_ms_fused": t_fused * 1e3,
+           "tflops_plain": (f_up + f_down) / t_plain / 1e12, "tflops_fused": (f_up + f_down) / t_fused / 1e12,
+           "outputs_bit_identical": identical, "clip_count": int(clip.item()),
+           "kernels_us_plain": {k: v * 1e6 for k, v in tp.items()},
+           "kernels_us_fused": {k: v * 1e6 for k, v in tf.items()},
+           "gemm_up_roofline": _gemm_roof(f_up, tp["gemm_up"], pk, False),
+           "gemm_down_roofline": _gemm_roof(f_down, tp["gemm_down"], pk, False),
+           "gemm_up_gelu_quant_roofline": _gemm_roof(f_up, tf["gemm_up_gelu_quant"], pk, False),
+           "quantizer_up_roofline": _quant_roof(M, K, tp["quant_up"], pk),
+           "quantizer_down_roofline": _quant_roof(M, N1, tp["quant_down"], pk),
+           "l2": "not flushed: every step's inputs and outputs exceed L2"}
+    if not args.no_cpu_baseline:
+        rows = 16
+        r1, d1 = _oracle_layer_rate(_bits(x), sg_x, _oracle_weights(w1), _bits(b1), rows)
+        r2, d2 = _oracle_layer_rate(_bits(g), sg_g, _oracle_weights(w2), _bits(b2), rows)
+        out["cpu_baseline"] = {"value": 2.0 * rows * (K * N1 + N1 * N2) / (d1 + d2) / 1e12, "unit": "TFLOPS",
+                               "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+                               "sample": f"{rows} token rows through both layers ({d1 + d2:.2f} s)"}
+    return out
+
+
+def measure_sweep_config(fh, S, dev, pk, args):
+    """Config 5: 42 blocks x {QKV 2688->8064, out 2688->2688, up 2688->10752,
+    down 10752->2688} = 168 layers back to back at 49152 tokens, each with its own
+    seeded weights, its own calibrated scale (amax over its 1000-batch stream)
+    and its own BF16 input (77 GB in all, resident in HBM), quantized per layer.
+    One step = the 168 quantize + GEMM pairs."""
+    import torch
+    sweep = S.workloads()["block_sweep"]
+    M = sweep[0].M
+    layers = []
+    shapes = {}
+    for layer in sweep:
+        x, sg_a = _dev_inputs(fh, S, layer, M, dev, calib=layer.n_calib)
+        wc, wsc, sg_w, b, w = _dev_weights(fh, S, layer, dev)
+        del w
+        key = (layer.K, layer.N)
+        if key not in shapes:  # codes and outputs are per shape: each layer overwrites its shape's buffers
+            shapes[key] = (*fh.empty_quantized(M, layer.K, device=dev),
+                           torch.empty((M, layer.N), dtype=torch.bfloat16, device=dev))
+        layers.append((layer, x, sg_a, wc, wsc, sg_w, b))
+    clip = torch.zeros(1, dtype=torch.int64, device=dev)
+    calls = []
+    for (layer, x, sg_a, wc, wsc, sg_w, b) in layers:
+        ac, asc, y = shapes[(layer.K, layer.N)]
+        tag = f"{layer.K}->{layer.N}"
+        calls.append(("quant " + tag, lambda x=x, sg_a=sg_a, ac=ac, asc=asc: fh.fh_quantize_act(x, sg_a, ac, asc, clip)))
+        calls.append(("gemm " + tag, lambda ac=ac, asc=asc, sg_a=sg_a, wc=wc, wsc=wsc, sg_w=sg_w, b=b, y=y:
+                      fh.fh_nvfp4_linear(ac, asc, sg_a, wc, wsc, sg_w, b, y)))
+    steps = 3
+    t, region = _time_calls(calls, steps, 3)
+    fh.fh_device_status()
+    nb = len(sweep) // 4
+    flops = {f"{l.K}->{l.N}": 2.0 * M * l.K * l.N * nb for l in sweep[:4]}
+    t_gemm = sum(v for k, v in t.items() if k.startswith("gemm"))
+    t_quant = sum(v for k, v in t.items() if k.startswith("quant"))
+    total_flops = sum(flops.values())
+    quant_bytes = QUANT_BYTES_PER_ELEM * M * sum(l.K for l in sweep)
+    # A 168-layer step runs for ~0.1 s of back-to-back GEMMs: the power-capped
+    # (sustained) GEMM figure is its denominator.
+    out = {"workload": f"block sweep {len(sweep)} layers at M={M}", "M": M, "layers": len(sweep), "steps": steps,
+           "step_ms": (t_gemm + t_quant) * 1e3, "tflops": total_flops / (t_gemm + t_quant) / 1e12,
+           "gemm_roofline": _gemm_roof(total_flops, t_gemm, pk, True),
+           "quantizer_roofline": {"bound": "hbm", "achieved": quant_bytes / t_quant / 1e9, "unit": "GB/s",
+                                  "peak": pk["hbm_gbs"], "frac": quant_bytes / t_quant / 1e9 / pk["hbm_gbs"],
+                                  "us": t_quant * 1e6},
+           "per_shape": {tag: {"gemm_us_per_layer": t["gemm " + tag] / nb * 1e6,
+                               "gemm_tflops": flops[tag] / t["gemm " + tag] / 1e12,
+                               "quant_us_per_layer": t["quant " + tag] / nb * 1e6,
+                               "quant_gbs": QUANT_BYTES_PER_ELEM * M * int(tag.split("->")[0]) * nb
+                               / t["quant " + tag] / 1e9} for tag in flops},
+           "clip_count": int(clip.item()), "inputs_gb": 2.0 * M * sum(l.K for l in sweep) / 1e9,
+           "l2": "not flushed: every layer's input (>= 264 MB) exceeds L2"}
+    if not args.no_cpu_baseline:
+        rows, secs, fl = 8, 0.0, 0.0
+        for (layer, x, sg_a, wc, wsc, sg_w, b) in layers[:4]:
+            w = S.weights_t(layer, dev).view(torch.bfloat16)
+            r, dt = _oracle_layer_rate(_bits(x[:rows]), sg_a, _oracle_weights(w), _bits(b), rows)
+            secs += dt
+            fl += 2.0 * rows * layer.K * layer.N
+        out["cpu_baseline"] = {"value": fl / secs / 1e12, "unit": "TFLOPS", "cores": len(os.sched_getaffinity(0)),
+                               "kind": "oracle", "sample": f"{rows} token rows through block 0's four layers "
+                                                           f"({secs:.2f} s)"}
+    del layers, shapes
+    torch.cuda.empty_cache()
+    return out
+
+
+def measure_configs(args, which=("tiny", "attn_proj", "ffn_pair", "block_sweep")):
+    import torch
+    import synthetic as S
+    import nvfp4_quantized_linear_fh_b200 as fh
+    dev = torch.device("cuda", torch.cuda.current_device())
+    pk = peaks()
+    out = {}
+    for name in which:
+        if name in ("tiny", "attn_proj"):
+            out[name] = measure_layer_config(name, fh, S, dev, pk, args)
+        elif name == "ffn_pair":
+            out[name] = measure_ffn_config(fh, S, dev, pk, args)
+        elif name == "block_sweep":
+            out[name] = measure_sweep_config(fh, S, dev, pk, args)
+        torch.cuda.empty_cache()
+    return out
 
 
 ATTN = {"heads": 21, "tokens": 4096, "d": 128}
@@ -632,10 +945,16 @@ def main():
     ap.add_argument("--M", type=int, default=WORKLOAD["M"],
                     help="token rows per GPU (profiling cases use fewer than the workload's 32768)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
-    ap.add_argument("--workload", default="qkv", choices=["qkv", "ffn", "attn", "adaln"],
-                    help="qkv: the headline line (fused QKV layer); ffn: the FFN block, fused vs unfused "
-                         "epilogue; attn: INT8 query/key quantization and attention scores; adaln: AdaLN "
-                         "basis projection")
+    ap.add_argument("--workload", default="qkv",
+                    choices=["qkv", "tiny", "attn_proj", "ffn_pair", "block_sweep", "ffn", "attn", "adaln"],
+                    help="qkv: the headline line (fused QKV layer), with the other four configurations in its "
+                         "'configs' object; tiny, attn_proj, ffn_pair, block_sweep: one of those configurations "
+                         "as a line of its own; ffn: the FFN block, fused vs unfused epilogue; attn: INT8 "
+                         "query/key quantization and attention scores; adaln: AdaLN basis projection")
+    ap.add_argument("--no-fused", action="store_true",
+                    help="skip timing the quantization fused into the GEMM (fh_nvfp4_linear_fused_quant)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="headline line only (skip the other four configurations)")
     ap.add_argument("--quick", action="store_true",
                     help="calibrate on the input batches only (setup shortcut for profiling cases)")
     args = ap.parse_args()
@@ -648,6 +967,12 @@ def main():
         return
     if args.workload == "adaln":
         bench_adaln(args)
+        return
+    if args.workload in ("tiny", "attn_proj", "ffn_pair", "block_sweep"):
+        import torch
+        torch.cuda.set_device(0)
+        cfg = measure_configs(args, (args.workload,))[args.workload]
+        print(json.dumps({"metric": METRIC, "workload": args.workload, "n_gpus": 1, "data": "synthetic", **cfg}))
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -736,11 +1061,28 @@ def main():
                         "4096-row chunks)"},
         "clocks": r["sampler"],
     }
+    if r["t_fused"]:
+        tf = statistics.mean(r["t_fused"])
+        line["fused_quant"] = {"call": "fh_nvfp4_linear_fused_quant (quantization inside the GEMM kernel)",
+                               "step_us": tf * 1e6, "tflops": r["flops"] / tf / 1e12,
+                               "vs_two_calls": (r["t_step"] / K_steps) / tf, "steps": len(r["t_fused"]),
+                               "output_identical_to_two_calls": True}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, dt, cores = cpu_baseline(r["x_bits"], r["w_bits"], r["b_bits"], r["sg_a"], r["sg_w"], CPU_SAMPLE_ROWS)
         line["cpu_baseline"] = {"value": v, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                                 "sample": f"first {CPU_SAMPLE_ROWS} token rows of the same layer (quantize the rows, "
                                           f"binary64 dequantized GEMM; weights quantized beforehand), {dt:.1f} s"}
+    if rank == 0:
+        # The FP4 tensor rate measured with the library's own probe (no memory
+        # traffic): the ceiling a block-scaled FP4 GEMM on this GPU can reach.
+        r_mma, r_cp = fp4_tensor_rate(False) / 1e12, fp4_tensor_rate(True) / 1e12
+        line["fp4_tensor_rate"] = {"mma_only": r_mma, "mma_with_scale_copies": r_cp, "unit": "TFLOP/s",
+                                   "how": "fh_selftest_mma_rate: one CTA pair per SM pair, 60000 rounds of four "
+                                          "256x256x64 kind::mxf4nvf4 MMAs from shared memory, best of 3"}
+        line["roofline"]["frac_of_measured_fp4_rate"] = achieved / r_mma
+    if rank == 0 and world == 1 and not args.no_configs and args.M == WORKLOAD["M"]:
+        # The other four configurations, measured after the headline's timed region.
+        line["configs"] = measure_configs(args)
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
