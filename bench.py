@@ -41,17 +41,28 @@ CPU_SAMPLE_ROWS = 64
 # DRAM bytes (read + write) of one GEMM launch on this workload, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
 # kernel source it was taken on (first 16 hex digits of its SHA-256).
-GEMM_TRAFFIC = {"bytes": 535824640, "source_sha256": "8e728c7adf255d1d"}
+GEMM_TRAFFIC = {"bytes": 576101376, "source_sha256": "4abe7c48fa84e050"}
+# The same for one quantizer launch inside the step (ncu --cache-control none,
+# so the L2 state the preceding GEMM left is kept); fh_quant.cu's hash.
+QUANT_TRAFFIC = {"bytes": 236669952, "source_sha256": "003adfc5d7f0ff56"}
 REF_ROWS = 16
 
 
-def gemm_traffic():
-    """Per-launch DRAM traffic of the GEMM if the kernel source is the one it was measured on."""
+def _traffic(record, source):
+    """A recorded per-launch DRAM traffic figure if the kernel source is the one it was measured on."""
     import hashlib
-    path = os.path.join(ROOT, "nvfp4_quantized_linear_fh_b200", "csrc", "fh_gemm.cu")
+    path = os.path.join(ROOT, "nvfp4_quantized_linear_fh_b200", "csrc", source)
     with open(path, "rb") as f:
         digest = hashlib.sha256(f.read()).hexdigest()[:16]
-    return GEMM_TRAFFIC["bytes"] if digest == GEMM_TRAFFIC["source_sha256"] else None
+    return record["bytes"] if digest == record["source_sha256"] else None
+
+
+def gemm_traffic():
+    return _traffic(GEMM_TRAFFIC, "fh_gemm.cu")
+
+
+def quant_traffic():
+    return _traffic(QUANT_TRAFFIC, "fh_quant.cu")
 
 
 def peaks():
@@ -922,7 +933,7 @@ def bench_adaln(args):
 
 # DRAM bytes (read + write) of one int8_scores_kernel launch on the workload
 # above, from an ncu capture; valid only for the kernel source it was taken on.
-ATTN_TRAFFIC = {"bytes": 1371787776, "source_sha256": "1c5edf861590e2be"}
+ATTN_TRAFFIC = {"bytes": 1371803392, "source_sha256": "8d69c5a712786aec"}
 
 
 def attn_traffic_valid():
@@ -1053,7 +1064,9 @@ def main():
                      "traffic_note": "bytes per launch, ncu dram__bytes_read.sum + dram__bytes_write.sum",
                      "algorithmic_bytes": gemm_bytes(r["M"], r["N"], r["K"])},
         "quantizer": {"kernel": "quantize_tiled_kernel", "bound": "hbm", "achieved": quant_gbs, "peak": pk["hbm_gbs"],
-                      "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"], "us": quant_mean * 1e6},
+                      "unit": "GB/s", "frac": quant_gbs / pk["hbm_gbs"], "us": quant_mean * 1e6,
+                      "traffic": quant_traffic() if r["M"] == WORKLOAD["M"] else None,
+                      "algorithmic_bytes": QUANT_BYTES_PER_ELEM * r["M"] * r["K"]},
         "gemm_us": gemm_mean * 1e6, "clip_count": r["clips"],
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "steps": r["e_steps"],
