@@ -37,7 +37,7 @@ METRIC = "NVFP4 linear TFLOPS (M×2688→N) and % of B200 FP4 peak; quantizer GB
 WORKLOAD = {"name": "qkv", "M": 32768, "K": 2688, "N": 8064}
 FP4_OVER_BF16 = 4.0        # nominal dense ratio 9 / 2.25 PFLOP/s
 QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16.0
-CPU_SAMPLE_ROWS = 64
+CPU_SAMPLE_ROWS = 4096   # about 10 s of the oracle on 16 host cores
 # DRAM bytes (read + write) of one GEMM launch on this workload, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
 # kernel source it was taken on (first 16 hex digits of its SHA-256).
