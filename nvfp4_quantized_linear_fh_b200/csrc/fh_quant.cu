@@ -440,26 +440,32 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
   if (threadIdx.x == 0 && cta_clips && p.clip) atomicAdd(p.clip, cta_clips);
 }
 
-// Tensor-core scale layout: each unit is a 128-row x 64-column tile of x
-// (16 KB), loaded by one 2-D tensor TMA whose out-of-range rows read as zero.
-// Thread t quantizes block t % 4 of tile row t / 4, so one unit yields exactly
-// one 512-byte scale atom (written by the unit's own threads, which lets L2
-// merge it) and 32-byte code segments; zero rows past M give the zero padding
-// scales the layout requires.
+// Tensor-core scale layout: each unit is a 128-row x 64 kG-column tile of x
+// (16 kG KB), loaded by one 2-D tensor TMA whose out-of-range rows read as
+// zero.  Thread t quantizes block t % 4 of every 64-column group of tile row
+// t / 4, so one unit yields exactly kG whole 512-byte scale atoms (written by
+// the unit's own threads, which lets L2 merge them) and 32-byte code
+// segments; zero rows past M give the zero padding scales the layout
+// requires.  The wider unit halves the TMA issues and barrier round trips per
+// byte; the ring keeps the same 96 KB.
 // kGelu: quantize GELU(x) instead of x (the FFN activation applied on the way,
 // with the same arithmetic as the stand-alone GELU kernel).
-template <bool kGelu>
+template <bool kGelu, int kG>
 __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_constant__ CUtensorMap tmx,
                                                                    const __grid_constant__ QuantParams p) {
+  // A unit is 128 rows x 64 kG columns (kG scale atoms); the ring holds the
+  // same 96 KB for either width.
+  constexpr int S = kQStages / kG;
+  constexpr int kUnitBytes = kQUnitBytes * kG;
   extern __shared__ __align__(128) uint8_t qsmem[];
   __shared__ QuantTable tab;
   __shared__ unsigned long long cta_clips;
   __shared__ int abort_flag_s;
   volatile int* abort_flag = &abort_flag_s;
   const uint32_t stage0 = q_smem_u32(qsmem);
-  const uint32_t bar0 = stage0 + kQStages * kQUnitBytes;
+  const uint32_t bar0 = stage0 + S * kUnitBytes;
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
-  auto empty_bar = [&](int st) { return bar0 + 8u * (kQStages + st); };
+  auto empty_bar = [&](int st) { return bar0 + 8u * (S + st); };
   {
     const uint4* src = reinterpret_cast<const uint4*>(&p.tab);
     uint4* dst = reinterpret_cast<uint4*>(&tab);
@@ -468,7 +474,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
   if (threadIdx.x == 0) {
     cta_clips = 0;
     abort_flag_s = 0;
-    for (int st = 0; st < kQStages; ++st) {
+    for (int st = 0; st < S; ++st) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full_bar(st)));
       asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty_bar(st)), "r"(kQConsumerWarps));
     }
@@ -483,17 +489,17 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t nb = p.K >> 4;
-  const int64_t katoms = nb >> 2;  // 64-column tiles per row block
+  const int64_t katoms = nb >> 2;  // 64-column tiles (scale atoms) per row block
   unsigned long long clips = 0;
-  // Unit u is tile (u / katoms, u % katoms); the CTA visits u = blockIdx.x,
-  // blockIdx.x + gridDim.x, ..., so both coordinates advance by constants
-  // (no division inside the loops).
-  const int ka = (int)katoms;
+  // Unit u is tile (u / ka, u % ka) of ka = K / (64 kG) units per row block;
+  // the CTA visits u = blockIdx.x, blockIdx.x + gridDim.x, ..., so both
+  // coordinates advance by constants (no division inside the loops).
+  const int ka = (int)katoms / kG;
   const int d_row = (int)(gridDim.x / ka), d_col = (int)(gridDim.x % ka);
   const int row0 = (int)(blockIdx.x / ka), col0 = (int)(blockIdx.x % ka);
 
   if (warp == kQConsumerWarps) {
-    // ===== producer: one tensor TMA per 128 x 64 tile =====
+    // ===== producer: one tensor TMA per 128 x 64 kG tile =====
     if (lane == 0) {
       const uint64_t read_once = evict_first_policy();
       int st = 0;
@@ -501,7 +507,7 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
       int tr = row0, tc = col0;
       for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
         if (!q_wait(empty_bar(st), ph ^ 1u, abort_flag)) break;
-        const int x0 = tc * 64, y0 = tr * 128;
+        const int x0 = tc * 64 * kG, y0 = tr * 128;
         tr += d_row;
         tc += d_col;
         if (tc >= ka) {
@@ -509,59 +515,63 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
           ++tr;
         }
         asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full_bar(st)),
-                     "r"((uint32_t)kQUnitBytes)
+                     "r"((uint32_t)kUnitBytes)
                      : "memory");
         asm volatile(
             "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-            " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(stage0 + st * kQUnitBytes),
+            " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(stage0 + st * kUnitBytes),
             "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(x0), "r"(y0), "r"(full_bar(st)), "l"(read_once)
             : "memory");
-        if (++st == kQStages) {
+        if (++st == S) {
           st = 0;
           ph ^= 1u;
         }
       }
-      for (int i = 0; i < kQStages; ++i) q_wait_drain(full_bar(i), (i < st) ? ph : (ph ^ 1u));
+      for (int i = 0; i < S; ++i) q_wait_drain(full_bar(i), (i < st) ? ph : (ph ^ 1u));
     }
   } else {
-    // ===== consumers: thread t quantizes block t % 4 of tile row t / 4 =====
+    // ===== consumers: thread t quantizes block t % 4 of every 64-column group of tile row t / 4 =====
     const int ctid = threadIdx.x;  // 0 .. 511
     const int r = ctid >> 2, j = ctid & 3;
-    const uint8_t* my_block = qsmem + 32 * ctid;
+    const uint8_t* my_block = qsmem + r * (128 * kG) + 32 * j;
+    const int word_off = (r & 31) * 16 + (r >> 5) * 4;  // the row's word in a scale atom
     int st = 0;
     uint32_t ph = 0;
     int tr = row0, tc = col0;
     for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
       if (!q_wait(full_bar(st), ph, abort_flag)) break;
       const int64_t m = (int64_t)tr * 128 + r;
-      const int64_t sg = (int64_t)tc * 4 + j;
+      const int cg0 = tc * kG;                                     // the unit's first 64-column group
+      const int64_t atom0 = (int64_t)tr * katoms + cg0;            // and its scale atom
       tr += d_row;
       tc += d_col;
       if (tc >= ka) {
         tc -= ka;
         ++tr;
       }
-      uint32_t sc = 0;
-      if (m < p.M) {
-        const uint8_t* blk = my_block + st * kQUnitBytes;
-        const uint4 q0 = *reinterpret_cast<const uint4*>(blk);
-        const uint4 q1 = *reinterpret_cast<const uint4*>(blk + 16);
-        uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-        if (kGelu) {
+#pragma unroll 1
+      for (int c = 0; c < kG; ++c) {
+        uint32_t sc = 0;
+        if (m < p.M) {
+          const uint8_t* blk = my_block + st * kUnitBytes + c * 128;
+          const uint4 q0 = *reinterpret_cast<const uint4*>(blk);
+          const uint4 q1 = *reinterpret_cast<const uint4*>(blk + 16);
+          uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+          if (kGelu) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) w[i] = gelu2_bits(w[i]);
+            for (int i = 0; i < 8; ++i) w[i] = gelu2_bits(w[i]);
+          }
+          sc = quantize_block(tab, p, w, m, (cg0 + c) * 4 + j, clips);
         }
-        sc = quantize_block(tab, p, w, m, sg, clips);
+        // Every row of the unit, padding rows included, writes its scales:
+        // lanes 4i..4i+3 (blocks 0..3 of row r) gather one word of the atom.
+        const uint32_t pair = sc | (__shfl_down_sync(0xFFFFFFFFu, sc, 1) << 8);
+        const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
+        if (j == 0) *reinterpret_cast<uint32_t*>(p.scales + (atom0 + c) * 512 + word_off) = word;
       }
-      // Every row of the unit, padding rows included, writes its scales: the
-      // unit's atom starts at byte 512 u; lanes 4i..4i+3 (blocks 0..3 of row
-      // r) gather one word at r0 * 16 + r1 * 4 (r = r0 + 32 r1).
-      const uint32_t pair = sc | (__shfl_down_sync(0xFFFFFFFFu, sc, 1) << 8);
-      const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
-      if (j == 0) *reinterpret_cast<uint32_t*>(p.scales + u * 512 + (r & 31) * 16 + (r >> 5) * 4) = word;
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
-      if (++st == kQStages) {
+      if (++st == S) {
         st = 0;
         ph ^= 1u;
       }
@@ -716,18 +726,21 @@ cudaError_t launch_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
     kernel<<<grid, kQThreads, kQSmem, s>>>(p);
     return cudaGetLastError();
   };
-  static DeviceTable cfg_ft, cfg_ff, cfg_t[2];
+  static DeviceTable cfg_ft, cfg_ff, cfg_t[4];
   if (tiled) {
-    // K % 64 == 0 here.  One unit per 128-row x 64-column tile.
+    // K % 64 == 0 here.  Units of 128 rows x 128 columns (two scale atoms)
+    // when K allows, else 128 x 64.
+    const int kg = (K % 128 == 0) ? 2 : 1;
     CUtensorMap tmx;
     if (!make_tensor_map_2d(&tmx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, (uint64_t)K, (uint64_t)M,
-                            (uint64_t)ldx * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+                            (uint64_t)ldx * 2, 64 * kg, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorNotSupported;
-    p.n_units = ((M + 127) / 128) * (K / 64);
+    p.n_units = ((M + 127) / 128) * (K / (64 * kg));
     const int64_t tw = p.n_units > 0 ? p.n_units : 1;
     const int tgrid = (int)(tw < 2 * (int64_t)sm_count() ? tw : 2 * (int64_t)sm_count());
-    auto kernel = gelu ? quantize_tiled_kernel<true> : quantize_tiled_kernel<false>;
-    cudaError_t e = configure(kernel, cfg_t[gelu ? 1 : 0]);
+    auto kernel = kg == 2 ? (gelu ? quantize_tiled_kernel<true, 2> : quantize_tiled_kernel<false, 2>)
+                          : (gelu ? quantize_tiled_kernel<true, 1> : quantize_tiled_kernel<false, 1>);
+    cudaError_t e = configure(kernel, cfg_t[(gelu ? 1 : 0) + 2 * (kg - 1)]);
     if (e != cudaSuccess) return e;
     kernel<<<tgrid, kQThreads, kQSmem, s>>>(tmx, p);
     return cudaGetLastError();
