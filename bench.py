@@ -37,14 +37,14 @@ METRIC = "NVFP4 linear TFLOPS (M×2688→N) and % of B200 FP4 peak; quantizer GB
 WORKLOAD = {"name": "qkv", "M": 32768, "K": 2688, "N": 8064}
 FP4_OVER_BF16 = 4.0        # nominal dense ratio 9 / 2.25 PFLOP/s
 QUANT_BYTES_PER_ELEM = 2.0 + 0.5 + 1.0 / 16.0
-CPU_SAMPLE_ROWS = 4096   # about 10 s of the oracle on 16 host cores
+CPU_SAMPLE_ROWS = 8192   # about 13 s of the oracle on 16 host cores
 # DRAM bytes (read + write) of one GEMM launch on this workload, from an ncu
 # capture (dram__bytes_read.sum + dram__bytes_write.sum); valid only for the
 # kernel source it was taken on (first 16 hex digits of its SHA-256).
 GEMM_TRAFFIC = {"bytes": 576101376, "source_sha256": "4abe7c48fa84e050"}
 # The same for one quantizer launch inside the step (ncu --cache-control none,
 # so the L2 state the preceding GEMM left is kept); fh_quant.cu's hash.
-QUANT_TRAFFIC = {"bytes": 236669952, "source_sha256": "003adfc5d7f0ff56"}
+QUANT_TRAFFIC = {"bytes": 231230336, "source_sha256": "d2928983a413a94e"}
 REF_ROWS = 16
 
 
