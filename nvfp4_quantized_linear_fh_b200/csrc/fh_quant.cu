@@ -219,6 +219,19 @@ __device__ __forceinline__ int64_t tiled_offset(int64_t m, int64_t s, int64_t ka
   return ((m >> 7) * katoms + (s >> 2)) * 512 + (m & 31) * 16 + ((m >> 5) & 3) * 4 + (s & 3);
 }
 
+// Quantize one loaded block: stores its 8 code bytes at dst, returns its scale
+// code and adds its clipped elements to clips.
+__device__ __forceinline__ uint32_t quantize_block_to(const QuantTable& tab, const QuantParams& p,
+                                                      const uint32_t* w, uint8_t* dst,
+                                                      unsigned long long& clips) {
+  uint32_t amax;
+  uint2 out;
+  const uint32_t c = quantize_block_codes(tab, p.inv6sg, w, amax, out);
+  *reinterpret_cast<uint2*>(dst) = out;
+  clips += block_clips(w, amax, p.clip_thr);
+  return c;
+}
+
 // Quantize one loaded block of row m: stores its 8 code bytes, returns its
 // scale code and adds its clipped elements to clips.
 __device__ __forceinline__ uint32_t quantize_block(const QuantTable& tab, const QuantParams& p,
@@ -256,7 +269,10 @@ constexpr int kQThreads = 32 * (kQConsumerWarps + 1);
 constexpr int kQStages = 6;
 constexpr int kQUnitElems = 8192;
 constexpr int kQUnitBytes = 2 * kQUnitElems;
-constexpr int kQSmem = kQStages * kQUnitBytes + 2 * 8 * kQStages + 64;
+// The tiled kernel stages each unit's scale atoms in shared memory (two
+// buffers per ring stage); the producer warp copies them out.
+constexpr int kQScaleStaging = 2 * kQStages * 512;
+constexpr int kQSmem = kQStages * kQUnitBytes + kQScaleStaging + 2 * 8 * kQStages + 64;
 static_assert(kQUnitElems / 16 == 32 * kQConsumerWarps, "one block per consumer thread per unit");
 
 __device__ unsigned int g_quant_error = 0;
@@ -443,11 +459,13 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(const __grid_consta
 // Tensor-core scale layout: each unit is a 128-row x 64 kG-column tile of x
 // (16 kG KB), loaded by one 2-D tensor TMA whose out-of-range rows read as
 // zero.  Thread t quantizes block t % 4 of every 64-column group of tile row
-// t / 4, so one unit yields exactly kG whole 512-byte scale atoms (written by
-// the unit's own threads, which lets L2 merge them) and 32-byte code
-// segments; zero rows past M give the zero padding scales the layout
-// requires.  The wider unit halves the TMA issues and barrier round trips per
-// byte; the ring keeps the same 96 KB.
+// t / 4, so one unit yields exactly kG whole 512-byte scale atoms and 32-byte
+// code segments; zero rows past M give the zero padding scales the layout
+// requires.  The consumers leave each scale byte in a shared-memory staging
+// buffer, and the producer warp, once the unit's stage is released, copies
+// the unit's atoms out with 16-byte stores (one scale store per lane instead
+// of gathers and a 4-byte store per row).  The wider unit halves the TMA
+// issues and barrier round trips per byte; the ring keeps the same 96 KB.
 // kGelu: quantize GELU(x) instead of x (the FFN activation applied on the way,
 // with the same arithmetic as the stand-alone GELU kernel).
 template <bool kGelu, int kG>
@@ -463,9 +481,14 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
   __shared__ int abort_flag_s;
   volatile int* abort_flag = &abort_flag_s;
   const uint32_t stage0 = q_smem_u32(qsmem);
-  const uint32_t bar0 = stage0 + S * kUnitBytes;
+  // Scale staging: buffer (st, b) holds the kG atoms of the unit in ring stage
+  // st whose ring phase bit is b.
+  const uint32_t sstage0 = stage0 + S * kUnitBytes;
+  auto scale_buf = [&](int st, uint32_t b) { return sstage0 + (uint32_t)((2 * st + (int)b) * kG * 512); };
+  const uint32_t bar0 = sstage0 + kQScaleStaging;
   auto full_bar = [&](int st) { return bar0 + 8u * st; };
   auto empty_bar = [&](int st) { return bar0 + 8u * (S + st); };
+  static_assert(2 * S * kG * 512 == kQScaleStaging, "staging size");
   {
     const uint4* src = reinterpret_cast<const uint4*>(&p.tab);
     uint4* dst = reinterpret_cast<uint4*>(&tab);
@@ -500,13 +523,37 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
 
   if (warp == kQConsumerWarps) {
     // ===== producer: one tensor TMA per 128 x 64 kG tile =====
-    if (lane == 0) {
+    {
       const uint64_t read_once = evict_first_policy();
       int st = 0;
       uint32_t ph = 0;
-      int tr = row0, tc = col0;
-      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-        if (!q_wait(empty_bar(st), ph ^ 1u, abort_flag)) break;
+      int tr = row0, tc = col0;  // the next unit to load
+      int sr = row0, sc = col0;  // the next unit whose scales go out
+      int64_t n = 0;             // units loaded
+      bool ok = true;
+      // Once the consumers are done with unit n - S (the wait for its ring
+      // stage), the warp copies its staged scale atoms (kG x 512 contiguous
+      // bytes) to global memory, 16 bytes per lane per step.
+      auto store_scales = [&](int stage, uint32_t b) {
+        const uint4* src = reinterpret_cast<const uint4*>(qsmem + (scale_buf(stage, b) - stage0));
+        uint4* dst = reinterpret_cast<uint4*>(p.scales + ((int64_t)sr * katoms + (int64_t)sc * kG) * 512);
+#pragma unroll
+        for (int i = 0; i < kG; ++i) dst[32 * i + lane] = src[32 * i + lane];
+        sr += d_row;
+        sc += d_col;
+        if (sc >= ka) {
+          sc -= ka;
+          ++sr;
+        }
+      };
+      for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x, ++n) {
+        if (!__all_sync(0xFFFFFFFFu, q_wait(empty_bar(st), ph ^ 1u, abort_flag))) {  // warp-uniform
+          ok = false;
+          break;
+        }
+        // Staging buffer (st, ph ^ 1) held unit n - S; buffer (st, ph), which
+        // unit n's consumers fill, was copied out S units ago.
+        if (n >= S) store_scales(st, ph ^ 1u);
         const int x0 = tc * 64 * kG, y0 = tr * 128;
         tr += d_row;
         tc += d_col;
@@ -514,35 +561,54 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
           tc -= ka;
           ++tr;
         }
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full_bar(st)),
-                     "r"((uint32_t)kUnitBytes)
-                     : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
-            " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(stage0 + st * kUnitBytes),
-            "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(x0), "r"(y0), "r"(full_bar(st)), "l"(read_once)
-            : "memory");
+        if (lane == 0) {
+          asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(full_bar(st)),
+                       "r"((uint32_t)kUnitBytes)
+                       : "memory");
+          asm volatile(
+              "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+              " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(stage0 + st * kUnitBytes),
+              "l"(reinterpret_cast<uint64_t>(&tmx)), "r"(x0), "r"(y0), "r"(full_bar(st)), "l"(read_once)
+              : "memory");
+        }
+        __syncwarp();
         if (++st == S) {
           st = 0;
           ph ^= 1u;
         }
       }
-      for (int i = 0; i < S; ++i) q_wait_drain(full_bar(i), (i < st) ? ph : (ph ^ 1u));
+      // The scales of the last S units, as their stages are released: the
+      // ring walk continues over S more positions without loading.
+      int tst = st;
+      uint32_t tph = ph;
+      for (int64_t k = n; ok && k < n + S; ++k) {
+        if (!__all_sync(0xFFFFFFFFu, q_wait(empty_bar(tst), tph ^ 1u, abort_flag))) break;
+        if (k >= S) store_scales(tst, tph ^ 1u);
+        if (++tst == S) {
+          tst = 0;
+          tph ^= 1u;
+        }
+      }
+      // The last load into each stage, from the position after the last loaded unit.
+      if (lane == 0)
+        for (int i = 0; i < S; ++i) q_wait_drain(full_bar(i), (i < st) ? ph : (ph ^ 1u));
+      __syncwarp();
     }
   } else {
     // ===== consumers: thread t quantizes block t % 4 of every 64-column group of tile row t / 4 =====
     const int ctid = threadIdx.x;  // 0 .. 511
     const int r = ctid >> 2, j = ctid & 3;
     const uint8_t* my_block = qsmem + r * (128 * kG) + 32 * j;
-    const int word_off = (r & 31) * 16 + (r >> 5) * 4;  // the row's word in a scale atom
+    const uint32_t scale_off = (uint32_t)((r & 31) * 16 + (r >> 5) * 4 + j);  // this block's byte in an atom
     int st = 0;
     uint32_t ph = 0;
     int tr = row0, tc = col0;
     for (int64_t u = blockIdx.x; u < p.n_units; u += gridDim.x) {
       if (!q_wait(full_bar(st), ph, abort_flag)) break;
       const int64_t m = (int64_t)tr * 128 + r;
-      const int cg0 = tc * kG;                                     // the unit's first 64-column group
-      const int64_t atom0 = (int64_t)tr * katoms + cg0;            // and its scale atom
+      const int cg0 = tc * kG;  // the unit's first 64-column group
+      uint8_t* crow = p.codes + m * (p.K >> 1) + 32 * cg0 + 8 * j;
+      const uint32_t sbuf = scale_buf(st, ph) + scale_off;
       tr += d_row;
       tc += d_col;
       if (tc >= ka) {
@@ -561,13 +627,10 @@ __global__ void __launch_bounds__(kQThreads) quantize_tiled_kernel(const __grid_
 #pragma unroll
             for (int i = 0; i < 8; ++i) w[i] = gelu2_bits(w[i]);
           }
-          sc = quantize_block(tab, p, w, m, (cg0 + c) * 4 + j, clips);
+          sc = quantize_block_to(tab, p, w, crow + 32 * c, clips);
         }
-        // Every row of the unit, padding rows included, writes its scales:
-        // lanes 4i..4i+3 (blocks 0..3 of row r) gather one word of the atom.
-        const uint32_t pair = sc | (__shfl_down_sync(0xFFFFFFFFu, sc, 1) << 8);
-        const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
-        if (j == 0) *reinterpret_cast<uint32_t*>(p.scales + (atom0 + c) * 512 + word_off) = word;
+        // Every row of the unit, padding rows included, stages its scales.
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(sbuf + 512u * c), "r"(sc) : "memory");
       }
       __syncwarp();
       if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(empty_bar(st)) : "memory");
