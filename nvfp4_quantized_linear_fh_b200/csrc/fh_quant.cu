@@ -27,12 +27,14 @@
 // threshold-compare path.  The block scale takes a converter candidate and
 // corrects it against the exact scale thresholds.
 //
-// Memory: a producer warp streams 16 KB units of x into a ring of shared-memory
-// stages; each of 512 consumer threads quantizes one 16-element block per unit
-// (one 32-byte shared-memory read, one 8-byte code store; four lanes gather
-// four consecutive block scales into one 4-byte store).  For the tensor-core
-// scale layout a unit is a 128-row x 64-column tile, so each unit writes
-// exactly one 512-byte scale atom; for row-major scales a unit is whole rows.
+// Memory: a producer warp streams units of x into a 96 KB ring of
+// shared-memory stages; each of 512 consumer threads quantizes one 16-element
+// block per 64 columns of the unit (one 32-byte shared-memory read, one 8-byte
+// code store).  For the tensor-core scale layout a unit is a 128-row x
+// 128-column tile (128 x 64 when K is an odd multiple of 64), whose whole
+// 512-byte scale atoms are staged in shared memory and copied out by the
+// producer warp; for row-major scales a unit is whole rows of 16 KB and four
+// lanes gather four consecutive block scales into one 4-byte store.
 // HBM-bound: 2.5625 bytes per element.
 #include <cuda_bf16.h>
 #include <math.h>
