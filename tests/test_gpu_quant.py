@@ -104,6 +104,20 @@ def test_tiny_workload_clip_counts():
     assert check_quantize(x, sg_unc, TILED) == 33
 
 
+# The tensor-core-layout quantizer runs 2 CTAs per SM over units of 128 rows x
+# 128 columns (3-stage ring) or, when K is an odd multiple of 64, 128 x 64
+# (6-stage ring); each unit's scale atoms leave through a staging buffer once
+# its ring stage is released.  On a 148-SM B200 these shapes give the CTAs 3,
+# 4 and 7 wide units, and 13 or 4 narrow ones: every ring position, the
+# end-of-loop stores and ragged row blocks.
+@pytest.mark.parametrize("M,K", [(3840, 2688), (5757, 2688), (11259, 2688), (11483, 2624), (2766, 2624)])
+def test_tiled_unit_counts(M, K):
+    x = S.random_bf16(("tiled-units", M, K), (M, K), 2.0)
+    sg = oracle.scale_from_amax(oracle.amax(x))
+    assert check_quantize(x, sg, TILED) == 0
+    assert check_quantize(x, sg / 64, TILED) > 0
+
+
 @pytest.mark.parametrize("name", ["attn_proj", "qkv"])
 def test_full_size_quantizer(name):
     layer = S.workloads()[name][0]
