@@ -146,7 +146,9 @@ def test_fused_192_wide_pair_form():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
 
 
-@pytest.mark.parametrize("M,K", [(100, 192), (129, 512), (300, 2688), (1, 64), (513, 10752)])
+# The last two shapes give the quantizer's CTAs 4 wide (128-column) and 13 narrow
+# (64-column) units each on a 148-SM B200, with ragged row blocks.
+@pytest.mark.parametrize("M,K", [(100, 192), (129, 512), (300, 2688), (1, 64), (513, 10752), (5757, 2688), (11483, 2624)])
 def test_gelu_quantize_matches_two_calls(M, K):
     """fh_gelu_quantize_act == fh_gelu_bf16 then fh_quantize_act, bit for bit
     (codes, every scale byte including padding rows, clip count)."""
